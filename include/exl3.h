@@ -1,0 +1,142 @@
+/*
+ * exl3.h -- C ABI of the B200 (sm_100a) EXL3 trellis-decoded matmul library.
+ *
+ * The operation: y = x . W_hat for fp16 activations x (m x k) and weights W_hat
+ * (k x n) that are never stored densely.  W_hat is kept as 16 x 16 tiles, each a
+ * K-bit-per-weight tail-biting bitshift trellis (K = 1..8) packed in uint16
+ * words, and is decoded on the fly through a procedural codebook.  The product
+ * is wrapped in two 128-point Hadamard rotations:
+ *
+ *     x' = H128(x .* suh) / sqrt(128)        (per 128-channel block of k)
+ *     y' = x' . W_hat                         (fp32 accumulation)
+ *     y  = svh .* H128(y') / sqrt(128)        (per 128-channel block of n)
+ *
+ * Sources (page titles):
+ *   [GEMM] "ExLlamaV3推理快的秘密: EXL3 GEMM内核与融合Viterbi编码CUDA实现剖析",
+ *          sections 先看结论 (conclusions), GEMM内核 (GEMM kernel: 128-point
+ *          Hadamard on the input fused with the dequantising matmul; the
+ *          codebook is one integer multiply + one lop3, no table),
+ *          小批量GEMV (small-batch GEMV for the decode phase, bandwidth bound),
+ *          Viterbi编码内核剖析 (16 x 16 tiles, tail-biting trellis, packed into
+ *          a 16-bit index sequence).
+ *   [OVW]  "为什么ExLlamaV3值得关注": EXL3 is a simplified QTIP variant with a
+ *          procedural codebook and a tail-biting trellis, 1..8 bits per weight.
+ *
+ * Data layout (the pages do not fix one; this library's convention):
+ *   x        m x k fp16, row-major.
+ *   trellis  uint16 [k/16][n/16][16*K]; tile (tk, tn) covers
+ *            W_hat[16tk + r][16tn + c], weight index i = 16 r + c.  The tile's
+ *            16K words are one big-endian bit string (bit 15 of word 0 first);
+ *            weight i's 16-bit state is the window of positions
+ *            [iK + K - 16, iK + K) taken modulo 256K (weight 0 wraps to the
+ *            stream's end), earliest position most significant.
+ *   codebook v = state * 89226354 + 64248484 (mod 2^32);
+ *            v = (v & 0x8fff8fff) ^ 0x3b603b60;
+ *            w = fp16(v >> 16) + fp16(v & 0xffff), bit patterns read as fp16,
+ *            sum rounded to nearest even.
+ *   suh      k fp16 (+-1 signs), svh n fp16 (signed per-channel scales).
+ *   y        m x n fp16, row-major.
+ *
+ * Conventions for every call:
+ *   - All array pointers are DEVICE memory owned by the caller, 16-byte
+ *     aligned; the library never allocates, frees or synchronises inside these
+ *     calls.  Work is enqueued asynchronously on `stream` (a cudaStream_t;
+ *     NULL = the legacy default stream).
+ *   - k and n must be multiples of 128; 1 <= K <= 8; y must not overlap x.
+ *   - Argument errors return EXL3_ERR_INVALID_ARG / EXL3_ERR_UNSUPPORTED /
+ *     EXL3_ERR_WORKSPACE before anything is launched.  A failed launch returns
+ *     EXL3_ERR_CUDA (the CUDA error is left for cudaGetLastError to report).
+ *   - Device-side waits are bounded.  A wait that runs out records a timeout
+ *     in the workspace's status word (read it with exl3_workspace_status) and
+ *     the kernel returns early; the output is then undefined.
+ *   - Calls are thread-safe; concurrent calls on different streams need
+ *     distinct workspaces.
+ */
+#ifndef EXL3_B200_H
+#define EXL3_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    EXL3_OK = 0,
+    EXL3_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, bad K          */
+    EXL3_ERR_UNSUPPORTED = 2, /* valid request this build does not handle (m > 16 for gemv) */
+    EXL3_ERR_WORKSPACE = 3,   /* workspace missing or smaller than *_workspace_size */
+    EXL3_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed               */
+    EXL3_ERR_TIMEOUT = 5      /* a bounded device wait ran out (see exl3_workspace_status) */
+} exl3_status;
+
+/* Static, human-readable name of a status code (never NULL). */
+const char *exl3_status_string(int status);
+
+/* Library version string, e.g. "exl3-b200 0.1 sm_100a". */
+const char *exl3_version(void);
+
+/*
+ * exl3_hadamard -- blockwise 128-point Hadamard rotation ([GEMM] section
+ * GEMM内核: the input is rotated by a 128-point Hadamard before the matmul).
+ *   y[r, 128b + i] = post[128b+i] * (1/sqrt(128)) * sum_j H[i][j] * x[r,128b+j] * pre[128b+j]
+ * with the Sylvester matrix H[i][j] = (-1)^popcount(i & j).
+ *   x, y      rows x cols fp16, row-major; cols % 128 == 0; y may equal x
+ *             (in place) but must not otherwise overlap it.
+ *   pre, post cols fp16 each, or NULL for all ones.
+ * Arithmetic in fp32, one fp16 rounding of the result.  rows == 0 is a no-op.
+ */
+exl3_status exl3_hadamard(const void *x, void *y, int64_t rows, int64_t cols,
+                          const void *pre, const void *post, void *stream);
+
+/*
+ * exl3_decode_tiles -- decode a whole trellis to dense fp16 weights, for
+ * checking ([GEMM] sections 先看结论 and GEMM内核: state -> fp16 through the
+ * procedural codebook; Viterbi编码内核剖析: tail-biting 16 x 16 tiles).
+ *   trellis   uint16 [k/16][n/16][16K] (layout above).
+ *   w         k x n fp16, row-major (output, caller-owned).
+ * Bit-exact: every weight equals the codebook value of its trellis state.
+ */
+exl3_status exl3_decode_tiles(const uint16_t *trellis, void *w, int64_t k, int64_t n, int K,
+                              void *stream);
+
+/*
+ * exl3_gemv -- the linear layer for small batches, 1 <= m <= 16 ([GEMM]
+ * section 小批量GEMV: in the decode phase the bottleneck is memory bandwidth).
+ * Arguments as in the layout above.  `workspace` (device memory, at least
+ * exl3_gemv_workspace_size bytes) holds fp32 split-k partial sums, arrival
+ * counters and a status word; it must be zero-filled ONCE after allocation
+ * (the kernels return the counters to zero themselves) and must not be shared
+ * by calls that can run concurrently.
+ */
+size_t exl3_gemv_workspace_size(int64_t m, int64_t k, int64_t n, int K);
+exl3_status exl3_gemv(const void *x, const uint16_t *trellis, const void *suh, const void *svh,
+                      void *y, int64_t m, int64_t k, int64_t n, int K, void *workspace,
+                      size_t workspace_bytes, void *stream);
+
+/*
+ * exl3_gemm -- the linear layer on the tensor cores (tcgen05 / TMEM), any
+ * m >= 1, tuned for m >= 64 ([GEMM] section GEMM内核: Hadamard rotation of the
+ * input, then the dequantising matmul; the kernel map picks tiles by shape).
+ * `workspace` (at least exl3_gemm_workspace_size bytes, zero-filled once after
+ * allocation) holds the rotated activations x' (m x k fp16) and a status
+ * word.  Same argument conventions as exl3_gemv.
+ */
+size_t exl3_gemm_workspace_size(int64_t m, int64_t k, int64_t n, int K);
+exl3_status exl3_gemm(const void *x, const uint16_t *trellis, const void *suh, const void *svh,
+                      void *y, int64_t m, int64_t k, int64_t n, int K, void *workspace,
+                      size_t workspace_bytes, void *stream);
+
+/*
+ * exl3_workspace_status -- read (synchronously, on `stream`) the status word a
+ * gemv/gemm call leaves in its workspace: EXL3_OK, or EXL3_ERR_TIMEOUT if a
+ * bounded device wait ran out.  `clear` != 0 resets it to EXL3_OK.
+ */
+exl3_status exl3_workspace_status(void *workspace, size_t workspace_bytes, int clear, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXL3_B200_H */

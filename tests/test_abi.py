@@ -1,0 +1,108 @@
+"""CPU-side checks of the C-ABI library: it builds, loads, exports every symbol
+the public headers declare, and rejects bad arguments before launching
+anything (no compute call is made here)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+from trellis_coded_bit_b200 import exl3
+
+HEADERS = sorted(glob.glob(os.path.join(ROOT, "include", "*.h")))
+
+
+def declared_functions():
+    names = []
+    for h in HEADERS:
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"\b(exl3_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_headers_declare_the_four_calls():
+    names = declared_functions()
+    for fn in ("exl3_hadamard", "exl3_decode_tiles", "exl3_gemv", "exl3_gemm"):
+        assert fn in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = exl3.load()
+    names = declared_functions()
+    assert set(names) == set(exl3.EXPORTED)
+    for name in names:
+        assert hasattr(lib, name), name  # ctypes raises AttributeError if not exported
+    assert exl3.library_path().startswith(os.path.join(ROOT, "trellis_coded_bit_b200"))
+
+
+def test_status_strings_and_version():
+    for code in range(6):
+        assert exl3.status_string(code).startswith("EXL3_")
+    assert "sm_100a" in exl3.version()
+
+
+def test_wait_limit_hook_roundtrip():
+    exl3.exl3_debug_set_wait_limit_ns(12345)
+    assert exl3.exl3_debug_wait_limit_ns() == 12345
+    exl3.exl3_debug_set_wait_limit_ns(0)
+    assert exl3.exl3_debug_wait_limit_ns() == 1_000_000_000
+
+
+# Fake, never-dereferenced device addresses: argument checks run before any
+# CUDA call, so these calls return without touching a GPU.
+A = 1 << 20        # 16-byte aligned
+B = 2 << 20
+C = 3 << 20
+D = 4 << 20
+E = 5 << 20
+MIS = A + 8        # misaligned
+
+
+def _gemv(fn, x=A, t=B, suh=C, svh=D, y=E, m=1, k=256, n=256, K=4, ws=None, wsb=1 << 20):
+    lib = exl3.load()
+    return getattr(lib, fn)(x, t, suh, svh, y, m, k, n, K, ws, wsb, None)
+
+
+@pytest.mark.parametrize("fn", ["exl3_gemv", "exl3_gemm"])
+def test_linear_argument_errors(fn):
+    inv = exl3.EXL3_ERR_INVALID_ARG
+    assert _gemv(fn, x=None) == inv
+    assert _gemv(fn, y=MIS) == inv
+    assert _gemv(fn, t=MIS) == inv
+    assert _gemv(fn, k=200) == inv          # not a multiple of 128
+    assert _gemv(fn, n=0) == inv
+    assert _gemv(fn, K=0) == inv
+    assert _gemv(fn, K=9) == inv
+    assert _gemv(fn, m=0) == inv
+    assert _gemv(fn, x=A, y=A) == inv       # y overlaps x
+
+
+def test_gemv_rejects_large_m_and_missing_workspace():
+    assert _gemv("exl3_gemv", m=17) == exl3.EXL3_ERR_UNSUPPORTED
+    assert _gemv("exl3_gemv", ws=None) == exl3.EXL3_ERR_WORKSPACE
+    assert _gemv("exl3_gemv", ws=A, wsb=16) == exl3.EXL3_ERR_WORKSPACE
+    assert _gemv("exl3_gemv", ws=MIS) == exl3.EXL3_ERR_WORKSPACE
+
+
+def test_workspace_sizes():
+    lib = exl3.load()
+    assert lib.exl3_gemv_workspace_size(1, 4096, 4096, 4) >= 256
+    assert lib.exl3_gemv_workspace_size(17, 4096, 4096, 4) == 0
+    assert lib.exl3_gemv_workspace_size(1, 100, 4096, 4) == 0
+    assert lib.exl3_gemm_workspace_size(2048, 8192, 28672, 3) >= 2048 * 8192 * 2
+
+
+def test_hadamard_and_decode_argument_errors():
+    lib = exl3.load()
+    inv = exl3.EXL3_ERR_INVALID_ARG
+    assert lib.exl3_hadamard(A, B, 4, 100, None, None, None) == inv
+    assert lib.exl3_hadamard(MIS, B, 4, 128, None, None, None) == inv
+    assert lib.exl3_hadamard(A, A + 64, 4, 128, None, None, None) == inv  # partial overlap
+    assert lib.exl3_hadamard(None, None, 0, 128, None, None, None) == exl3.EXL3_OK  # empty
+    assert lib.exl3_decode_tiles(A, B, 16, 16, 0, None) == inv
+    assert lib.exl3_decode_tiles(A, B, 24, 16, 4, None) == inv
+    assert lib.exl3_decode_tiles(None, B, 16, 16, 4, None) == inv
+    assert lib.exl3_workspace_status(None, 0, 0, None) == exl3.EXL3_ERR_WORKSPACE

@@ -1,0 +1,559 @@
+// gemm.cu -- exl3_gemm: y = svh .* H(H(x .* suh) . W_hat) on the fifth-
+// generation tensor cores (tcgen05.mma, accumulators in TMEM), with W_hat
+// decoded from the trellis into shared memory on the fly (EXL3 GEMM kernel
+// article, section GEMM内核: the input is Hadamard-rotated, then the kernel
+// reads the quantised weights, decodes them with the procedural codebook and
+// multiplies, in one pass; the kernel map picks tile shapes).
+//
+// B200 design (the pages' consumer-GPU kernel is prior art, not a blueprint):
+//   1. A rotation pass computes x' = H(x .* suh)/sqrt(128) in fp32 and writes
+//      it as fp16 directly in the tensor core's canonical K-major, 128-byte
+//      swizzled tile layout ([m/128][k/64] tiles of 128 rows x 64 channels,
+//      16 KB each), so one 1-D bulk copy moves one A tile into shared memory.
+//   2. The main kernel: one CTA per 256 x 256 output tile (two M=128 tiles
+//      that share every decoded B stage), 18 warps:
+//        warp 0   producer: per 64-channel k block, bulk-copies the two A
+//                 tiles and the 4 trellis tile rows (16 tiles each) into a
+//                 stage, completing on an mbarrier (no multicast);
+//        warp 1   allocates 512 TMEM columns; one lane issues
+//                 tcgen05.mma.cta_group::1.kind::f16 (M=128, N=256, K=16,
+//                 fp32 accumulate, A K-major, B MN-major) and commits to
+//                 mbarriers that free the stage / signal the epilogue;
+//        warps 2..17 decode: lane u of a warp decodes run u (8 consecutive
+//                 output channels of one input channel) of one trellis tile,
+//                 sums the codebook halves in fp16 (RNE, the exact W_hat) and
+//                 stores the 16-byte run into the MN-major 128-byte-swizzled
+//                 B stage; fence.proxy.async then an mbarrier arrive.
+//      After the k loop, warps 2..5 (one TMEM lane quarter each) read the
+//      accumulators with tcgen05.ld, apply the 128-point output rotation as
+//      H4 (x) H32 (32-point butterflies in registers, a TMEM round trip, then
+//      the 4-point stage), scale by svh/sqrt(128) and store fp16 y.
+//   All waits are bounded; a timeout is recorded in the workspace status word
+//   and every role drains its in-flight copies / MMAs before the CTA exits.
+#include <cuda_fp16.h>
+
+#include "exl3_device.cuh"
+#include "exl3_host.h"
+
+namespace exl3 {
+
+constexpr int kBM = 128;             // rows per MMA tile (TMEM lanes)
+constexpr int kMT = 2;               // M tiles per CTA sharing one decoded B
+constexpr int kBN = 256;             // output channels per CTA (MMA N)
+constexpr int kBK = 64;              // input channels per stage
+constexpr int kDecWarps = 16;
+constexpr int kGemmThreads = 32 * (2 + kDecWarps);
+constexpr int kATileBytes = kBM * kBK * 2;   // 16 KB
+constexpr int kBTileBytes = kBK * kBN * 2;   // 32 KB
+constexpr int kTmemCols = kMT * kBN;         // 512
+
+__host__ __device__ constexpr int gemm_trellis_stage_bytes(int K)
+{
+    return (kBK / 16) * (kBN / 16) * 32 * K;  // 4 tile rows x 16 tiles
+}
+
+__host__ __device__ constexpr int gemm_stage_bytes(int K)
+{
+    return kMT * kATileBytes + kBTileBytes + ((gemm_trellis_stage_bytes(K) + 1023) & ~1023);
+}
+
+__host__ __device__ constexpr int gemm_stages(int K)
+{
+    return (220 * 1024) / gemm_stage_bytes(K) >= 3 ? 3 : 2;
+}
+
+__host__ __device__ constexpr int gemm_smem_bytes(int K)
+{
+    return 1024 /* alignment slack */ + 1024 /* barriers etc. */ + gemm_stages(K) * gemm_stage_bytes(K);
+}
+
+// ----------------------------------------------------- tcgen05 wrappers ---
+
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
+                     smem_addr(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before()
+{
+    asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after()
+{
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate)
+{
+    asm volatile(
+        "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
+                     smem_addr(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+
+#define EXL3_TMEM_LD32(taddr, v)                                                                          \
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14," \
+                 "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"          \
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),     \
+                   "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), \
+                   "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),           \
+                   "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),           \
+                   "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])            \
+                 : "r"(taddr))
+
+#define EXL3_TMEM_ST32(taddr, v)                                                                          \
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13," \
+                 "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n" ::"r"(   \
+                     taddr),                                                                               \
+                 "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),   \
+                 "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),          \
+                 "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),        \
+                 "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),        \
+                 "r"(v[29]), "r"(v[30]), "r"(v[31])                                                        \
+                 : "memory")
+
+#define EXL3_TMEM_LD8(taddr, v)                                                                           \
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"                \
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),     \
+                   "=r"(v[7])                                                                              \
+                 : "r"(taddr))
+
+// Wait for tcgen05.ld to land; the 32 destination registers are tied to the
+// wait so that no use of them can be scheduled before it.
+#define EXL3_TMEM_WAIT_LD32(v)                                                                            \
+    asm volatile("tcgen05.wait::ld.sync.aligned;\n"                                                       \
+                 : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]),     \
+                   "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]), "+r"(v[12]), "+r"(v[13]), \
+                   "+r"(v[14]), "+r"(v[15]), "+r"(v[16]), "+r"(v[17]), "+r"(v[18]), "+r"(v[19]),           \
+                   "+r"(v[20]), "+r"(v[21]), "+r"(v[22]), "+r"(v[23]), "+r"(v[24]), "+r"(v[25]),           \
+                   "+r"(v[26]), "+r"(v[27]), "+r"(v[28]), "+r"(v[29]), "+r"(v[30]), "+r"(v[31])            \
+                 :                                                                                         \
+                 : "memory")
+
+__device__ __forceinline__ void tmem_wait_st()
+{
+    asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
+}
+
+// Shared-memory matrix descriptor: 128-byte swizzle, sm_100 format.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo)
+{
+    return (uint64_t)((saddr >> 4) & 0x3fffu) | ((uint64_t)((lbo >> 4) & 0x3fffu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3fffu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor, kind::f16: D f32, A f16 K-major, B f16 MN-major.
+__host__ __device__ constexpr uint32_t gemm_idesc()
+{
+    return (1u << 4) | (0u << 7) | (0u << 10) | (0u << 15) | (1u << 16) | ((uint32_t)(kBN >> 3) << 17) |
+           ((uint32_t)(kBM >> 4) << 24);
+}
+
+// 32-point Sylvester Hadamard on 32 fp32 values held by one thread.
+__device__ __forceinline__ void fwht32(float (&v)[32])
+{
+#pragma unroll
+    for (int h = 1; h < 32; h <<= 1)
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            if ((i & h) == 0) {
+                const float a = v[i], b = v[i + h];
+                v[i] = a + b;
+                v[i + h] = a - b;
+            }
+}
+
+// -------------------------------------------------------- rotation pass ---
+
+// x'[r, :] = H(x[r, :] .* suh)/sqrt(128) written in the tiled, swizzled A
+// layout: tile (r/128, c/64), 128-byte row r%128, 16-byte chunk ((c%64)/8) ^ (r%8).
+__global__ void __launch_bounds__(256) rotate_tiled_kernel(const __half *__restrict__ x,
+                                                           const __half *__restrict__ suh,
+                                                           unsigned char *__restrict__ xt, int m, int k)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t blocks = (int64_t)m * (k / 128);
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < blocks; w += warps) {
+        const int r = (int)(w / (k / 128));
+        const int blk = (int)(w - (int64_t)r * (k / 128));
+        const int c = blk * 128 + lane * 4;
+        const uint2 raw = *reinterpret_cast<const uint2 *>(x + (int64_t)r * k + c);
+        const uint2 sr = *reinterpret_cast<const uint2 *>(suh + c);
+        const __half2 *xv = reinterpret_cast<const __half2 *>(&raw);
+        const __half2 *sv = reinterpret_cast<const __half2 *>(&sr);
+        float v[4] = {__low2float(xv[0]) * __low2float(sv[0]), __high2float(xv[0]) * __high2float(sv[0]),
+                      __low2float(xv[1]) * __low2float(sv[1]), __high2float(xv[1]) * __high2float(sv[1])};
+        warp_fwht128(v);
+        const float s = 0.08838834764831845f;
+        __half2 o0 = __floats2half2_rn(v[0] * s, v[1] * s);
+        __half2 o1 = __floats2half2_rn(v[2] * s, v[3] * s);
+        const int kb = c >> 6, chunk = (c & 63) >> 3, within = c & 7;
+        const int64_t tile = (int64_t)(r >> 7) * (k >> 6) + kb;
+        const int row = r & 127;
+        unsigned char *dst = xt + tile * kATileBytes + row * 128 + ((chunk ^ (row & 7)) << 4) + within * 2;
+        uint2 out;
+        out.x = *reinterpret_cast<uint32_t *>(&o0);
+        out.y = *reinterpret_cast<uint32_t *>(&o1);
+        *reinterpret_cast<uint2 *>(dst) = out;
+    }
+}
+
+// ------------------------------------------------------------ main kernel ---
+
+struct GemmParams {
+    const unsigned char *xt;   // tiled x'
+    const uint16_t *trellis;
+    const __half *svh;
+    __half *y;
+    int m, k, n;
+    uint32_t *status;
+    uint64_t wait_ns;
+};
+
+template <int K>
+__global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmParams p)
+{
+    constexpr int S = gemm_stages(K);
+    constexpr int kStage = gemm_stage_bytes(K);
+    constexpr int kTrellisBytes = gemm_trellis_stage_bytes(K);
+    constexpr int kTileRowBytes = (kBN / 16) * 32 * K;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint64_t *full_a = reinterpret_cast<uint64_t *>(smem);  // A + trellis landed
+    uint64_t *full_b = full_a + S;                            // B decoded
+    uint64_t *empty = full_b + S;                             // MMAs done with the stage
+    uint64_t *acc_full = empty + S;
+    uint64_t *drain = acc_full + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    unsigned char *stages = smem + 1024;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tiles_n = p.n / kBN;
+    const int tm = blockIdx.x / tiles_n, tn = blockIdx.x - (blockIdx.x / tiles_n) * tiles_n;
+    const int m0 = tm * kBM * kMT;
+    const int kblocks = p.k / kBK;
+    const int mt_count = (p.m - m0) > kBM ? kMT : 1;  // skip an M tile that is all padding
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full_a[s], 1);
+            mbar_init(&full_b[s], kDecWarps);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1)
+        tmem_alloc(tmem_slot, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ producer ---
+        if (lane == 0) {
+            int issued = 0;
+            for (int kb = 0; kb < kblocks; ++kb) {
+                const int s = kb % S;
+                const uint32_t ph = (uint32_t)(kb / S) & 1u;
+                if (!mbar_wait(&empty[s], ph ^ 1u, p.wait_ns)) {
+                    record_timeout(p.status);
+                    *abort_flag = 1;
+                    break;
+                }
+                unsigned char *st = stages + s * kStage;
+                mbar_arrive_expect_tx(&full_a[s], (uint32_t)(mt_count * kATileBytes + kTrellisBytes));
+                for (int mt = 0; mt < mt_count; ++mt) {
+                    const int64_t tile = (int64_t)((m0 >> 7) + mt) * kblocks + kb;
+                    bulk_g2s(st + mt * kATileBytes, p.xt + tile * kATileBytes, kATileBytes, &full_a[s]);
+                }
+                unsigned char *tr = st + kMT * kATileBytes + kBTileBytes;
+                for (int r = 0; r < kBK / 16; ++r) {
+                    const int64_t row = (int64_t)kb * (kBK / 16) + r;
+                    const uint16_t *src = p.trellis + (row * (p.n / 16) + (int64_t)tn * (kBN / 16)) * 16 * K;
+                    bulk_g2s(tr + r * kTileRowBytes, src, kTileRowBytes, &full_a[s]);
+                }
+                issued = kb + 1;
+            }
+            for (int kb = (issued > S ? issued - S : 0); kb < issued; ++kb)
+                if (!mbar_wait(&full_a[kb % S], (uint32_t)(kb / S) & 1u, kDefaultWaitNs))
+                    record_timeout(p.status);
+        }
+    } else if (warp == 1) {
+        // ----------------------------------------------------- MMA issuer ---
+        if (lane == 0) {
+            const uint32_t idesc = gemm_idesc();
+            bool ok = true;
+            int kb = 0;
+            for (; kb < kblocks; ++kb) {
+                const int s = kb % S;
+                const uint32_t ph = (uint32_t)(kb / S) & 1u;
+                if (!mbar_wait(&full_a[s], ph, p.wait_ns) || !mbar_wait(&full_b[s], ph, p.wait_ns)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a0 = smem_addr(stages + s * kStage);
+                const uint32_t b0 = a0 + kMT * kATileBytes;
+#pragma unroll
+                for (int kk = 0; kk < kBK / 16; ++kk) {
+                    const uint64_t bdesc = smem_desc(b0 + kk * 2048, 8192, 1024);
+                    for (int mt = 0; mt < mt_count; ++mt) {
+                        const uint64_t adesc = smem_desc(a0 + mt * kATileBytes + kk * 32, 16, 1024);
+                        mma_f16_ss(tmem + (uint32_t)(mt * kBN), adesc, bdesc, idesc, (kb | kk) ? 1u : 0u);
+                    }
+                }
+                mma_commit(&empty[s]);
+            }
+            if (ok) {
+                mma_commit(acc_full);
+            } else {
+                record_timeout(p.status);
+                *abort_flag = 1;
+            }
+            // make sure no MMA is still writing TMEM when the CTA tears down
+            mma_commit(drain);
+            if (!mbar_wait(drain, 0, kDefaultWaitNs))
+                record_timeout(p.status);
+        }
+    } else {
+        // ------------------------------------------------------- decoders ---
+        const int dw = warp - 2;
+        for (int kb = 0; kb < kblocks; ++kb) {
+            const int s = kb % S;
+            const uint32_t ph = (uint32_t)(kb / S) & 1u;
+            if (!warp_wait(&full_a[s], ph, p.wait_ns)) {
+                if (lane == 0) {
+                    record_timeout(p.status);
+                    *abort_flag = 1;
+                }
+                break;
+            }
+            unsigned char *st = stages + s * kStage;
+            unsigned char *bt = st + kMT * kATileBytes;
+            const unsigned char *tr = bt + kBTileBytes;
+#pragma unroll 1
+            for (int j = 0; j < (kBK / 16) * (kBN / 16) / kDecWarps; ++j) {
+                const int tile = j * kDecWarps + dw;      // 0 .. 63 within the stage
+                const int trow = tile / (kBN / 16), tcol = tile - trow * (kBN / 16);
+                const uint32_t *tw = reinterpret_cast<const uint32_t *>(tr + tile * 32 * K);
+                uint32_t sts[8];
+                if constexpr (K <= 6) {
+                    run_states<K, 8>(tw, lane * 8 * K, sts);
+                } else {
+                    uint32_t lo[4], hi[4];
+                    run_states<K, 4>(tw, lane * 8 * K, lo);
+                    run_states<K, 4>(tw, lane * 8 * K + 4 * K, hi);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        sts[q] = lo[q];
+                        sts[4 + q] = hi[q];
+                    }
+                }
+                uint32_t out[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    __half2 h2 = __halves2half2(codebook_weight(sts[2 * q]), codebook_weight(sts[2 * q + 1]));
+                    out[q] = *reinterpret_cast<uint32_t *>(&h2);
+                }
+                // run (row u/2, half u%2) -> k row, first output channel of the 8
+                const int kr = trow * 16 + (lane >> 1);
+                const int n0 = tcol * 16 + (lane & 1) * 8;
+                unsigned char *dst = bt + ((n0 >> 6) * (kBK / 8) + (kr >> 3)) * 1024 + (kr & 7) * 128 +
+                                     ((((n0 & 63) >> 3) ^ (kr & 7)) << 4);
+                *reinterpret_cast<uint4 *>(dst) = make_uint4(out[0], out[1], out[2], out[3]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&full_b[s]);
+        }
+
+        // ------------------------------------------------------ epilogue ---
+        if (dw < 4) {
+            const int quarter = warp & 3;  // TMEM lanes this warp may access
+            const bool have = warp_wait(acc_full, 0, p.wait_ns);
+            if (!have) {
+                if (lane == 0)
+                    record_timeout(p.status);
+            } else if (!*abort_flag) {
+                tc_fence_after();
+                const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+                for (int mt = 0; mt < mt_count; ++mt) {
+                    const int row = m0 + mt * kBM + quarter * 32 + lane;
+                    for (int hb = 0; hb < kBN / 128; ++hb) {
+                        const uint32_t col0 = (uint32_t)(mt * kBN + hb * 128);
+                        // 32-point butterflies on each 32-column chunk, written back to TMEM
+#pragma unroll 1
+                        for (int c = 0; c < 4; ++c) {
+                            uint32_t r[32];
+                            EXL3_TMEM_LD32(tmem + lane_base + col0 + 32 * c, r);
+                            EXL3_TMEM_WAIT_LD32(r);
+                            float v[32];
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                v[i] = __uint_as_float(r[i]);
+                            fwht32(v);
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                r[i] = __float_as_uint(v[i]);
+                            EXL3_TMEM_ST32(tmem + lane_base + col0 + 32 * c, r);
+                            tmem_wait_st();
+                        }
+                        // 4-point stage across the chunks, scale, fp16, store
+#pragma unroll 1
+                        for (int o = 0; o < 4; ++o) {
+                            uint32_t u[32];  // [chunk c][8 columns]
+                            EXL3_TMEM_LD8(tmem + lane_base + col0 + 0 + 8 * o, (u + 0));
+                            EXL3_TMEM_LD8(tmem + lane_base + col0 + 32 + 8 * o, (u + 8));
+                            EXL3_TMEM_LD8(tmem + lane_base + col0 + 64 + 8 * o, (u + 16));
+                            EXL3_TMEM_LD8(tmem + lane_base + col0 + 96 + 8 * o, (u + 24));
+                            EXL3_TMEM_WAIT_LD32(u);
+                            if (row < p.m) {
+#pragma unroll
+                                for (int c = 0; c < 4; ++c) {
+                                    const int ncol = tn * kBN + hb * 128 + 32 * c + 8 * o;
+                                    const uint4 sv4 = *reinterpret_cast<const uint4 *>(p.svh + ncol);
+                                    const __half2 *sv = reinterpret_cast<const __half2 *>(&sv4);
+                                    uint32_t pk[4];
+#pragma unroll
+                                    for (int e = 0; e < 8; e += 2) {
+                                        float z[2];
+#pragma unroll
+                                        for (int d = 0; d < 2; ++d) {
+                                            const float a0 = __uint_as_float(u[0 + e + d]);
+                                            const float a1 = __uint_as_float(u[8 + e + d]);
+                                            const float a2 = __uint_as_float(u[16 + e + d]);
+                                            const float a3 = __uint_as_float(u[24 + e + d]);
+                                            const float s01 = a0 + a1, d01 = a0 - a1, s23 = a2 + a3,
+                                                        d23 = a2 - a3;
+                                            // H4 row c: c=0 (+,+,+,+) c=1 (+,-,+,-) c=2 (+,+,-,-) c=3 (+,-,-,+)
+                                            z[d] = c == 0 ? s01 + s23 : c == 1 ? d01 + d23 : c == 2 ? s01 - s23 : d01 - d23;
+                                        }
+                                        const float s = 0.08838834764831845f;
+                                        __half2 h = __floats2half2_rn(z[0] * s * __low2float(sv[e >> 1]),
+                                                                      z[1] * s * __high2float(sv[e >> 1]));
+                                        pk[e >> 1] = *reinterpret_cast<uint32_t *>(&h);
+                                    }
+                                    *reinterpret_cast<uint4 *>(p.y + (int64_t)row * p.n + ncol) =
+                                        make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                                }
+                            }
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------- dispatch ---
+
+static size_t gemm_xt_bytes(int64_t m, int64_t k)
+{
+    const int64_t mp = (m + kBM * kMT - 1) / (kBM * kMT) * (kBM * kMT);
+    return (size_t)mp * (size_t)k * 2;
+}
+
+template <int K>
+static exl3_status launch_gemm_t(const GemmParams &p, cudaStream_t stream)
+{
+    constexpr int smem = gemm_smem_bytes(K);
+    auto kern = gemm_kernel<K>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return EXL3_ERR_CUDA;
+    const int tiles = ((p.m + kBM * kMT - 1) / (kBM * kMT)) * (p.n / kBN);
+    kern<<<tiles, kGemmThreads, smem, stream>>>(p);
+    return launch_status();
+}
+
+}  // namespace exl3
+
+extern "C" size_t exl3_gemm_workspace_size(int64_t m, int64_t k, int64_t n, int K)
+{
+    if (m < 1 || k < 128 || n < 256 || (k % 128) || (n % 256) || K < 1 || K > 8)
+        return 0;
+    return 1024 + exl3::gemm_xt_bytes(m, k);
+}
+
+extern "C" exl3_status exl3_gemm(const void *x, const uint16_t *trellis, const void *suh,
+                                 const void *svh, void *y, int64_t m, int64_t k, int64_t n, int K,
+                                 void *workspace, size_t workspace_bytes, void *stream)
+{
+    using namespace exl3;
+    const exl3_status st = check_linear_args(x, trellis, suh, svh, y, m, k, n, K);
+    if (st != EXL3_OK)
+        return st;
+    if (n % kBN)
+        return EXL3_ERR_UNSUPPORTED;
+    if (!workspace || !aligned16(workspace) || workspace_bytes < exl3_gemm_workspace_size(m, k, n, K))
+        return EXL3_ERR_WORKSPACE;
+    cudaStream_t s = (cudaStream_t)stream;
+    unsigned char *ws = (unsigned char *)workspace;
+    unsigned char *xt = ws + 1024;  // 1024-byte aligned relative to a 16-byte aligned base? see below
+    // the tiled x' buffer must be 16-byte aligned for the bulk copies
+    int64_t rot_grid = (m * (k / 128) + 7) / 8;
+    if (rot_grid > 148 * 16)
+        rot_grid = 148 * 16;
+    rotate_tiled_kernel<<<(unsigned)rot_grid, 256, 0, s>>>((const __half *)x, (const __half *)suh, xt, (int)m,
+                                                           (int)k);
+    if (launch_status() != EXL3_OK)
+        return EXL3_ERR_CUDA;
+    GemmParams p;
+    p.xt = xt;
+    p.trellis = trellis;
+    p.svh = (const __half *)svh;
+    p.y = (__half *)y;
+    p.m = (int)m;
+    p.k = (int)k;
+    p.n = (int)n;
+    p.status = (uint32_t *)ws;
+    p.wait_ns = wait_limit_ns();
+    switch (K) {
+    case 1: return launch_gemm_t<1>(p, s);
+    case 2: return launch_gemm_t<2>(p, s);
+    case 3: return launch_gemm_t<3>(p, s);
+    case 4: return launch_gemm_t<4>(p, s);
+    case 5: return launch_gemm_t<5>(p, s);
+    case 6: return launch_gemm_t<6>(p, s);
+    case 7: return launch_gemm_t<7>(p, s);
+    default: return launch_gemm_t<8>(p, s);
+    }
+}

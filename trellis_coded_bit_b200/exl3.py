@@ -1,0 +1,182 @@
+"""Thin ctypes binding of the EXL3 B200 C ABI (include/exl3.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of libexl3_b200.so.  PyTorch supplies device memory and streams.
+There is no CPU fallback: if the library cannot be built or loaded, or no
+CUDA device is present, these functions raise.
+"""
+import ctypes
+import os
+import threading
+
+import torch
+
+from . import build as _build
+
+EXL3_OK = 0
+EXL3_ERR_INVALID_ARG = 1
+EXL3_ERR_UNSUPPORTED = 2
+EXL3_ERR_WORKSPACE = 3
+EXL3_ERR_CUDA = 4
+EXL3_ERR_TIMEOUT = 5
+
+# Every symbol the public headers declare.
+EXPORTED = ["exl3_status_string", "exl3_version", "exl3_hadamard", "exl3_decode_tiles",
+            "exl3_gemv_workspace_size", "exl3_gemv", "exl3_gemm_workspace_size", "exl3_gemm",
+            "exl3_workspace_status", "exl3_debug_set_wait_limit_ns", "exl3_debug_wait_limit_ns"]
+
+_lib = None
+_lock = threading.Lock()
+
+
+class Exl3Error(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__("%s: %s" % (where, status_string(status)))
+
+
+def library_path():
+    return _build.LIB
+
+
+def load(build_if_needed=True):
+    """Load (building first if the sources are newer) the shared library."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        path = _build.build() if build_if_needed else _build.LIB
+        if not os.path.exists(path):
+            raise RuntimeError("EXL3 CUDA library not found at %s" % path)
+        lib = ctypes.CDLL(path)
+        vp, i64, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
+        ci = ctypes.c_int
+        lib.exl3_status_string.argtypes = [ci]
+        lib.exl3_status_string.restype = ctypes.c_char_p
+        lib.exl3_version.argtypes = []
+        lib.exl3_version.restype = ctypes.c_char_p
+        lib.exl3_hadamard.argtypes = [vp, vp, i64, i64, vp, vp, vp]
+        lib.exl3_hadamard.restype = ci
+        lib.exl3_decode_tiles.argtypes = [vp, vp, i64, i64, ci, vp]
+        lib.exl3_decode_tiles.restype = ci
+        for name in ("exl3_gemv_workspace_size", "exl3_gemm_workspace_size"):
+            getattr(lib, name).argtypes = [i64, i64, i64, ci]
+            getattr(lib, name).restype = sz
+        for name in ("exl3_gemv", "exl3_gemm"):
+            getattr(lib, name).argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, ci, vp, sz, vp]
+            getattr(lib, name).restype = ci
+        lib.exl3_workspace_status.argtypes = [vp, sz, ci, vp]
+        lib.exl3_workspace_status.restype = ci
+        lib.exl3_debug_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+        lib.exl3_debug_set_wait_limit_ns.restype = None
+        lib.exl3_debug_wait_limit_ns.argtypes = []
+        lib.exl3_debug_wait_limit_ns.restype = ctypes.c_uint64
+        _lib = lib
+        return lib
+
+
+def status_string(status):
+    return load().exl3_status_string(int(status)).decode()
+
+
+def version():
+    return load().exl3_version().decode()
+
+
+def _check(status, where):
+    if status != EXL3_OK:
+        raise Exl3Error(status, where)
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev(t, dtype, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError("%s must be a CUDA tensor" % name)
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _ptr_or_none(t, dtype, name):
+    return None if t is None else _dev(t, dtype, name)
+
+
+# ----------------------------------------------------------------- calls ---
+
+def exl3_hadamard(x, y=None, pre=None, post=None, stream=None):
+    """y = H128(x .* pre)/sqrt(128) .* post, blockwise over the last dimension."""
+    rows, cols = x.shape
+    if y is None:
+        y = torch.empty_like(x)
+    _check(load().exl3_hadamard(_dev(x, torch.float16, "x"), _dev(y, torch.float16, "y"), rows, cols,
+                                _ptr_or_none(pre, torch.float16, "pre"),
+                                _ptr_or_none(post, torch.float16, "post"), _stream(stream)),
+           "exl3_hadamard")
+    return y
+
+
+def exl3_decode_tiles(trellis, k, n, K, w=None, stream=None):
+    """Dense k x n fp16 weights decoded from a [k/16, n/16, 16K] uint16 trellis."""
+    if w is None:
+        w = torch.empty((k, n), dtype=torch.float16, device=trellis.device)
+    _check(load().exl3_decode_tiles(_dev(trellis, torch.uint16, "trellis"), _dev(w, torch.float16, "w"),
+                                    k, n, K, _stream(stream)), "exl3_decode_tiles")
+    return w
+
+
+def exl3_gemv_workspace_size(m, k, n, K):
+    return int(load().exl3_gemv_workspace_size(m, k, n, K))
+
+
+def exl3_gemm_workspace_size(m, k, n, K):
+    return int(load().exl3_gemm_workspace_size(m, k, n, K))
+
+
+def new_workspace(nbytes, device=None):
+    """Zero-filled workspace buffer (uint8) of at least nbytes, 256-byte aligned."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8,
+                       device=device if device is not None else "cuda")
+
+
+def _linear(fn, name, x, trellis, suh, svh, K, y, workspace, stream):
+    m, k = x.shape
+    n = svh.numel()
+    if y is None:
+        y = torch.empty((m, n), dtype=torch.float16, device=x.device)
+    if workspace is None:
+        raise ValueError("%s needs a workspace (see new_workspace / *_workspace_size)" % name)
+    _check(fn(_dev(x, torch.float16, "x"), _dev(trellis, torch.uint16, "trellis"),
+              _dev(suh, torch.float16, "suh"), _dev(svh, torch.float16, "svh"),
+              _dev(y, torch.float16, "y"), m, k, n, int(K), _dev(workspace, torch.uint8, "workspace"),
+              workspace.numel(), _stream(stream)), name)
+    return y
+
+
+def exl3_gemv(x, trellis, suh, svh, K, y=None, workspace=None, stream=None):
+    """y = svh .* H(H(x .* suh) W_hat) for 1 <= m <= 16 (memory-bound path)."""
+    return _linear(load().exl3_gemv, "exl3_gemv", x, trellis, suh, svh, K, y, workspace, stream)
+
+
+def exl3_gemm(x, trellis, suh, svh, K, y=None, workspace=None, stream=None):
+    """The same layer on the tensor cores, any m (tuned for m >= 64)."""
+    return _linear(load().exl3_gemm, "exl3_gemm", x, trellis, suh, svh, K, y, workspace, stream)
+
+
+def exl3_workspace_status(workspace, clear=False, stream=None):
+    """Status word of a gemv/gemm workspace (synchronises the stream)."""
+    return int(load().exl3_workspace_status(_dev(workspace, torch.uint8, "workspace"), workspace.numel(),
+                                            1 if clear else 0, _stream(stream)))
+
+
+def exl3_debug_set_wait_limit_ns(ns):
+    load().exl3_debug_set_wait_limit_ns(int(ns))
+
+
+def exl3_debug_wait_limit_ns():
+    return int(load().exl3_debug_wait_limit_ns())
