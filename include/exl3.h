@@ -129,6 +129,23 @@ exl3_status exl3_gemm(const void *x, const uint16_t *trellis, const void *suh, c
                       size_t workspace_bytes, void *stream);
 
 /*
+ * Launch options, process-wide (default 0).
+ *
+ * EXL3_LAUNCH_PDL -- launch exl3_gemv / exl3_gemm kernels with programmatic
+ *   dependent launch (CUDA programmatic stream serialization): a kernel may
+ *   start while the preceding kernel in the stream is still finishing, and
+ *   it begins streaming its WEIGHT operands (trellis, suh, svh) at once; all
+ *   other reads (x, the workspace) and every write wait until the preceding
+ *   kernel has completed and its writes are visible.  Enable it only when the
+ *   weights are not written by the kernel launched immediately before on the
+ *   same stream (true for inference with loaded weights).  Has no effect on
+ *   results.
+ */
+#define EXL3_LAUNCH_PDL 1u
+void exl3_set_launch_flags(unsigned flags);
+unsigned exl3_launch_flags(void);
+
+/*
  * exl3_workspace_status -- read (synchronously, on `stream`) the status word a
  * gemv/gemm call leaves in its workspace: EXL3_OK, or EXL3_ERR_TIMEOUT if a
  * bounded device wait ran out.  `clear` != 0 resets it to EXL3_OK.

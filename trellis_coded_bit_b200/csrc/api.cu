@@ -12,6 +12,12 @@
 namespace exl3 {
 
 static std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};
+static std::atomic<unsigned> g_launch_flags{0u};
+
+unsigned launch_flags()
+{
+    return g_launch_flags.load(std::memory_order_relaxed);
+}
 
 uint64_t wait_limit_ns()
 {
@@ -62,4 +68,14 @@ extern "C" void exl3_debug_set_wait_limit_ns(uint64_t ns)
 extern "C" uint64_t exl3_debug_wait_limit_ns(void)
 {
     return exl3::wait_limit_ns();
+}
+
+extern "C" void exl3_set_launch_flags(unsigned flags)
+{
+    exl3::g_launch_flags.store(flags & EXL3_LAUNCH_PDL, std::memory_order_relaxed);
+}
+
+extern "C" unsigned exl3_launch_flags(void)
+{
+    return exl3::launch_flags();
 }

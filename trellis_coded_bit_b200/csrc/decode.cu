@@ -1,10 +1,14 @@
 // decode.cu -- exl3_decode_tiles: trellis -> dense fp16 weights (the checking
-// path).  Each warp decodes one 16x16 tile; lane u decodes the run of 8
-// consecutive weights of tile row u/2, columns 8(u%2) .. 8(u%2)+7, i.e. the
-// stream bits [64uK/8 ... ) -- every run starts on a byte.  The 8 weights are
-// written as one 16-byte store.  Sources: EXL3 GEMM kernel article, sections
-// 先看结论 / GEMM内核 (procedural codebook) and Viterbi编码内核剖析 (16x16
-// tail-biting tiles packed as a 16-bit sequence).
+// path).  Sources: EXL3 GEMM kernel article, sections 先看结论 / GEMM内核
+// (procedural codebook) and Viterbi编码内核剖析 (16x16 tail-biting tiles
+// packed as a 16-bit sequence).
+//
+// It runs the same row decoder as the GEMM's decoder warps (row_weights_f16:
+// compile-time bit windows, codebook, fp16 RNE sum), so its bit-exact parity
+// also pins the hot paths' window arithmetic.  A warp takes 4 tiles; in two
+// passes (even rows, then odd rows, so that a pass's lanes share the row
+// parity) lane l decodes row 2(l%8)+pass of tile l/8: 16 weights written as
+// two 16-byte stores.
 #include <cuda_fp16.h>
 
 #include "exl3_device.cuh"
@@ -12,45 +16,42 @@
 
 namespace exl3 {
 
+template <int K, int PAR>
+__device__ __forceinline__ void decode_one_row(const uint32_t *tile, int row, const Codebook &cb, __half *dst)
+{
+    uint32_t raw[RowSpan<K, PAR>::N32];
+    load_row<K, PAR>(tile, row, raw);
+    uint32_t w[8];
+    row_weights_f16<K, RowSpan<K, PAR>::P>(raw, cb, w);
+    reinterpret_cast<uint4 *>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    reinterpret_cast<uint4 *>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+}
+
 template <int K>
 __global__ void __launch_bounds__(256) decode_tiles_kernel(const uint16_t *__restrict__ trellis,
                                                            __half *__restrict__ w, int64_t k,
-                                                           int64_t n)
+                                                           int64_t n, const Codebook cb)
 {
     const int lane = threadIdx.x & 31;
     const int64_t tn_count = n >> 4;
     const int64_t tiles = (k >> 4) * tn_count;
+    const int64_t groups = (tiles + 3) >> 2;  // 4 tiles per warp
     const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < tiles;
-         t += warps) {
+    for (int64_t gi = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); gi < groups;
+         gi += warps) {
+        const int64_t t = gi * 4 + (lane >> 3);
+        if (t >= tiles)
+            continue;
         const uint32_t *tile = reinterpret_cast<const uint32_t *>(trellis + t * 16 * K);
-        const int row = lane >> 1, half = lane & 1;
-        uint32_t s[8];
-        if constexpr (K <= 6) {
-            run_states<K, 8>(tile, lane * 8 * K, s);
-        } else {
-            uint32_t a[4], b[4];
-            run_states<K, 4>(tile, lane * 8 * K, a);
-            run_states<K, 4>(tile, lane * 8 * K + 4 * K, b);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                s[j] = a[j];
-                s[4 + j] = b[j];
-            }
-        }
-        uint32_t out[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            __half2 h2 = __halves2half2(codebook_weight(s[2 * j]), codebook_weight(s[2 * j + 1]));
-            out[j] = *reinterpret_cast<uint32_t *>(&h2);
-        }
         const int64_t tk = t / tn_count, tn = t - tk * tn_count;
-        __half *dst = w + (tk * 16 + row) * n + tn * 16 + half * 8;
-        *reinterpret_cast<uint4 *>(dst) = make_uint4(out[0], out[1], out[2], out[3]);
+        const int row0 = 2 * (lane & 7);
+        __half *base = w + (tk * 16) * n + tn * 16;
+        decode_one_row<K, 0>(tile, row0, cb, base + (int64_t)row0 * n);
+        decode_one_row<K, 1>(tile, row0 + 1, cb, base + (int64_t)(row0 + 1) * n);
     }
 }
 
-typedef void (*decode_fn)(const uint16_t *, __half *, int64_t, int64_t);
+typedef void (*decode_fn)(const uint16_t *, __half *, int64_t, int64_t, const Codebook);
 
 static decode_fn decode_table(int K)
 {
@@ -78,10 +79,11 @@ extern "C" exl3_status exl3_decode_tiles(const uint16_t *trellis, void *w, int64
         return EXL3_ERR_INVALID_ARG;
     if (ranges_overlap(trellis, (size_t)(k * n * K / 8), w, (size_t)(k * n * 2)))
         return EXL3_ERR_INVALID_ARG;
-    const int64_t tiles = (k / 16) * (n / 16);
-    int64_t grid = (tiles + 7) / 8;
+    const int64_t groups = ((k / 16) * (n / 16) + 3) / 4;
+    int64_t grid = (groups + 7) / 8;
     if (grid > 148 * 16)
         grid = 148 * 16;
-    decode_table(K)<<<(unsigned)grid, 256, 0, (cudaStream_t)stream>>>(trellis, (__half *)w, k, n);
+    decode_table(K)<<<(unsigned)grid, 256, 0, (cudaStream_t)stream>>>(trellis, (__half *)w, k, n,
+                                                                    codebook_constants());
     return launch_status();
 }

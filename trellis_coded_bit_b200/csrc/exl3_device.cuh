@@ -31,6 +31,19 @@ __device__ __forceinline__ uint64_t global_ns()
     return t;
 }
 
+// Programmatic dependent launch: wait for the preceding grid in the stream
+// to complete (no-op when the launch did not allow overlap) / let the next
+// grid start launching.
+__device__ __forceinline__ void grid_dep_wait()
+{
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void grid_dep_launch()
+{
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
 // ------------------------------------------------------------ bit stream ---
 
 // Words are stored little-endian, the bit string is big-endian per word: the
@@ -41,63 +54,139 @@ __device__ __forceinline__ uint32_t be32(uint32_t raw)
     return __byte_perm(raw, 0u, 0x1032);
 }
 
-// 64 stream bits starting at bit position `pos` (earliest bit = bit 63) of a
-// tile held as 8K 32-bit words at `tile`.  pos may be in [-32, 256K); the read
-// wraps cyclically (tail-biting).
-template <int K>
-__device__ __forceinline__ uint64_t read_bits64(const uint32_t *tile, int pos)
+// ------------------------------------------------------------ tile rows ---
+//
+// A tile row holds 16 weights = 16K bits = exactly K words, so row r starts at
+// word rK.  Its states need the row's K words plus the word before (the
+// prefix; for row 0 the tile's last word -- the tail-biting wrap).  The
+// 32-bit loads covering those K + 1 words start on a half-word position P:
+// P = 1 when the prefix word is the upper half of the first load, P = 0 when
+// it is the lower half.  P depends only on K and the row's parity, so callers
+// that process rows of one parity at a time get compile-time layouts.
+
+template <int K, int PAR>
+struct RowSpan {
+    static constexpr int P = (PAR == 0) ? 1 : ((K & 1) ? 0 : 1);
+    static constexpr int N32 = (P + K + 2) / 2;  // 32-bit loads covering K + 1 words
+};
+
+// Loads the words of tile row `row` (of parity PAR) from a tile of 8K 32-bit
+// words.  raw[0] holds the prefix word; the loads are read-only (nc) and as
+// wide as the row's alignment allows.
+template <int K, int PAR, int N>
+__device__ __forceinline__ void load_row(const uint32_t *__restrict__ tile, int row, uint32_t (&raw)[N])
 {
-    constexpr int kWords32 = 8 * K;  // 32-bit words per tile
-    constexpr int kBits = 256 * K;
-    if (pos < 0)
-        pos += kBits;
-    int q0 = pos >> 5;
-    const int o = pos & 31;
-    int q1 = q0 + 1;
-    if (q1 >= kWords32)
-        q1 -= kWords32;
-    int q2 = q1 + 1;
-    if (q2 >= kWords32)
-        q2 -= kWords32;
-    const uint32_t a = be32(tile[q0]);
-    const uint32_t b = be32(tile[q1]);
-    const uint32_t c = be32(tile[q2]);
-    const uint32_t hi = __funnelshift_l(b, a, o);
-    const uint32_t lo = __funnelshift_l(c, b, o);
-    return ((uint64_t)hi << 32) | lo;
+    constexpr int P = RowSpan<K, PAR>::P;
+    constexpr int N32 = RowSpan<K, PAR>::N32;
+    static_assert(N >= N32, "raw buffer too small");
+    const int first = (row * K - 1) >> 1;  // floor; -1 for row 0
+    raw[0] = __ldg(tile + (first < 0 ? 8 * K - 1 : first));
+    if constexpr (K == 4 && P == 1) {
+        const uint2 v = __ldg(reinterpret_cast<const uint2 *>(tile + first + 1));
+        raw[1] = v.x;
+        raw[2] = v.y;
+    } else if constexpr (K == 8 && P == 1) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(tile + first + 1));
+        raw[1] = v.x;
+        raw[2] = v.y;
+        raw[3] = v.z;
+        raw[4] = v.w;
+    } else {
+#pragma unroll
+        for (int i = 1; i < N32; ++i)
+            raw[i] = __ldg(tile + first + i);
+    }
 }
 
-// States of N consecutive weights of one tile row, the first of which starts
-// its own K bits at stream bit `start` (a multiple of 8: every run of 8
-// weights starts on a byte).  N * K + 16 - K must fit the 64 bits read.
-template <int K, int N>
-__device__ __forceinline__ void run_states(const uint32_t *tile, int start, uint32_t (&s)[N])
+// The 16 states of a tile row from its loaded words.  Word W[-1] (prefix) is
+// at half-word position P, W[i] at P + 1 + i.  Weight j's window ends at row
+// bit e = (j + 1) K: it lies in V = W[a-1]:W[a] (a = e / 16) shifted right by
+// c = 16 - e % 16; c = 16 is the word W[a-1] itself.  Every window is one
+// byte permute (with zero fill), from V or from V pre-shifted by c % 8 bits;
+// all selectors are compile-time constants.
+template <int K, int P, int N>
+__device__ __forceinline__ void row_states(const uint32_t (&raw)[N], uint32_t (&s)[16])
 {
-    static_assert((N - 1) * K + 16 <= 64, "run does not fit one 64-bit read");
-    const uint64_t r = read_bits64<K>(tile, start - (16 - K));
 #pragma unroll
-    for (int j = 0; j < N; ++j)
-        s[j] = (uint32_t)(r >> (48 - j * K)) & 0xffffu;
+    for (int j = 0; j < 16; ++j) {
+        const int e = (j + 1) * K;
+        const int a = e >> 4;
+        const int c = 16 - (e & 15);
+        const int pos = P + a;  // half-word position of W[a-1]
+        if (c == 16) {
+            s[j] = __byte_perm(raw[pos >> 1], 0u, (pos & 1) ? 0x4432u : 0x4410u);
+        } else {
+            const uint32_t v = (pos & 1) ? __byte_perm(raw[pos >> 1], raw[(pos >> 1) + 1], 0x3254u)
+                                         : __byte_perm(raw[pos >> 1], 0u, 0x1032u);
+            const int r = c & 7, cb = c >> 3;
+            const uint32_t sel = 0x4400u | ((uint32_t)(cb + 1) << 4) | (uint32_t)cb;
+            s[j] = __byte_perm(r ? (v >> r) : v, 0u, sel);
+        }
+    }
+}
+
+// Same as load_row for a tile held in shared memory (plain loads).
+template <int K, int PAR, int N>
+__device__ __forceinline__ void load_row_plain(const uint32_t *tile, int row, uint32_t (&raw)[N])
+{
+    constexpr int N32 = RowSpan<K, PAR>::N32;
+    static_assert(N >= N32, "raw buffer too small");
+    const int first = (row * K - 1) >> 1;
+    raw[0] = tile[first < 0 ? 8 * K - 1 : first];
+#pragma unroll
+    for (int i = 1; i < N32; ++i)
+        raw[i] = tile[first + i];
 }
 
 // ------------------------------------------------------------- codebook ---
 
-// The procedural codebook's 32-bit word for a state: one multiply-add and one
-// mask/xor (EXL3 GEMM kernel article, sections 先看结论 and GEMM内核: "one
-// integer multiply + one lop3, no table lookup").  Its two 16-bit halves are
-// fp16 bit patterns whose sum is the weight.
-__device__ __forceinline__ uint32_t codebook_word(uint32_t state)
+// The procedural codebook's constants.  Kernels receive them as launch
+// parameters and keep them in registers: a SASS instruction encodes at most
+// one 32-bit immediate, so with literal constants the mask/xor would split
+// into two logic ops; from registers it is one IMAD plus one LOP3 per weight,
+// the "one integer multiply + one lop3" of the EXL3 GEMM kernel article
+// (sections 先看结论 and GEMM内核).
+constexpr uint32_t kCbMul = 89226354u;
+constexpr uint32_t kCbAdd = 64248484u;
+constexpr uint32_t kCbMask = 0x8fff8fffu;
+constexpr uint32_t kCbXor = 0x3b603b60u;
+
+struct Codebook {
+    uint32_t mul, add, mask, xr;
+};
+
+__host__ __device__ inline Codebook codebook_constants()
 {
-    uint32_t v = state * 89226354u + 64248484u;
-    return (v & 0x8fff8fffu) ^ 0x3b603b60u;
+    return Codebook{kCbMul, kCbAdd, kCbMask, kCbXor};
 }
 
-// The weight itself: the two halves added in fp16, round-to-nearest-even.
-__device__ __forceinline__ __half codebook_weight(uint32_t state)
+// The codebook's 32-bit word for a state; its two 16-bit halves are fp16 bit
+// patterns whose sum is the weight.
+__device__ __forceinline__ uint32_t codebook_word(uint32_t state, const Codebook &cb)
 {
-    const uint32_t v = codebook_word(state);
-    const __half2 h = *reinterpret_cast<const __half2 *>(&v);
-    return __hadd(__low2half(h), __high2half(h));
+    const uint32_t v = state * cb.mul + cb.add;
+    return (v & cb.mask) ^ cb.xr;
+}
+
+
+// The exact fp16 weights of one tile row (row_states + codebook, the halves
+// added in fp16 with round-to-nearest-even), packed as 8 half2: out[j] holds
+// the weights of columns 2j and 2j+1.
+template <int K, int P, int N>
+__device__ __forceinline__ void row_weights_f16(const uint32_t (&raw)[N], const Codebook &cb,
+                                                uint32_t (&out)[8])
+{
+    uint32_t s[16];
+    row_states<K, P>(raw, s);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const uint32_t v0 = codebook_word(s[2 * j], cb);
+        const uint32_t v1 = codebook_word(s[2 * j + 1], cb);
+        const uint32_t lo = __byte_perm(v0, v1, 0x5410u);  // low halves of both words
+        const uint32_t hi = __byte_perm(v0, v1, 0x7632u);  // high halves of both words
+        __half2 w = __hadd2(*reinterpret_cast<const __half2 *>(&lo), *reinterpret_cast<const __half2 *>(&hi));
+        out[j] = *reinterpret_cast<uint32_t *>(&w);
+    }
 }
 
 // ------------------------------------------------------------ hadamard ----

@@ -23,6 +23,31 @@ inline bool ranges_overlap(const void *a, size_t an, const void *b, size_t bn)
 // Bound of device-side waits in nanoseconds (see exl3_debug.h).
 uint64_t wait_limit_ns();
 
+// Process-wide launch options (EXL3_LAUNCH_PDL).
+unsigned launch_flags();
+
+// Launches `kernel` with the library's launch options: with EXL3_LAUNCH_PDL
+// the launch allows programmatic dependent launch (the kernel itself calls
+// griddepcontrol.wait before touching anything but weights).
+template <typename... Args>
+inline cudaError_t launch_kernel(void (*kernel)(Args...), dim3 grid, dim3 block, size_t smem,
+                                 cudaStream_t stream, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    if (launch_flags() & EXL3_LAUNCH_PDL) {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 inline exl3_status launch_status()
 {
     return cudaPeekAtLastError() == cudaSuccess ? EXL3_OK : EXL3_ERR_CUDA;

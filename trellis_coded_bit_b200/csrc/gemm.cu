@@ -197,6 +197,8 @@ __global__ void __launch_bounds__(256) rotate_tiled_kernel(const __half *__restr
                                                            unsigned char *__restrict__ xt, int m, int k)
 {
     const int lane = threadIdx.x & 31;
+    grid_dep_wait();    // x is produced by the preceding kernel
+    grid_dep_launch();  // the GEMM kernel may set up (barriers, TMEM) meanwhile
     const int64_t blocks = (int64_t)m * (k / 128);
     const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
     for (int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < blocks; w += warps) {
@@ -224,6 +226,29 @@ __global__ void __launch_bounds__(256) rotate_tiled_kernel(const __half *__restr
     }
 }
 
+// Decodes tile row `row` of a shared-memory tile (stage tile row trow, column
+// tcol) to exact fp16 weights and stores its 16 values as two 16-byte chunks of
+// the MN-major, 128-byte-swizzled B stage: input channel kr is a row of an
+// 8-row x 64-column atom (atoms of 8 k rows at 1024 B, 64-column groups at
+// 8192 B), chunk (n % 64) / 8 lands at chunk position ((n % 64) / 8) ^ (kr % 8).
+template <int K, int PAR>
+__device__ __forceinline__ void decode_row_to_b(const uint32_t *tile, int row, const Codebook &cb,
+                                                unsigned char *bt, int trow, int tcol)
+{
+    uint32_t raw[RowSpan<K, PAR>::N32];
+    load_row_plain<K, PAR>(tile, row, raw);
+    uint32_t w[8];
+    row_weights_f16<K, RowSpan<K, PAR>::P>(raw, cb, w);
+    const int kr = trow * 16 + row;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int n0 = tcol * 16 + h * 8;
+        unsigned char *dst = bt + ((n0 >> 6) * (kBK / 8) + (kr >> 3)) * 1024 + (kr & 7) * 128 +
+                             ((((n0 & 63) >> 3) ^ (kr & 7)) << 4);
+        *reinterpret_cast<uint4 *>(dst) = make_uint4(w[4 * h], w[4 * h + 1], w[4 * h + 2], w[4 * h + 3]);
+    }
+}
+
 // ------------------------------------------------------------ main kernel ---
 
 struct GemmParams {
@@ -234,6 +259,7 @@ struct GemmParams {
     int m, k, n;
     uint32_t *status;
     uint64_t wait_ns;
+    Codebook cb;
 };
 
 template <int K>
@@ -278,6 +304,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmParams 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    grid_dep_wait();  // x' comes from the rotation kernel just before
 
     if (warp == 0) {
         // ------------------------------------------------------ producer ---
@@ -362,36 +389,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmParams 
             unsigned char *st = stages + s * kStage;
             unsigned char *bt = st + kMT * kATileBytes;
             const unsigned char *tr = bt + kBTileBytes;
-#pragma unroll 1
-            for (int j = 0; j < (kBK / 16) * (kBN / 16) / kDecWarps; ++j) {
-                const int tile = j * kDecWarps + dw;      // 0 .. 63 within the stage
-                const int trow = tile / (kBN / 16), tcol = tile - trow * (kBN / 16);
-                const uint32_t *tw = reinterpret_cast<const uint32_t *>(tr + tile * 32 * K);
-                uint32_t sts[8];
-                if constexpr (K <= 6) {
-                    run_states<K, 8>(tw, lane * 8 * K, sts);
-                } else {
-                    uint32_t lo[4], hi[4];
-                    run_states<K, 4>(tw, lane * 8 * K, lo);
-                    run_states<K, 4>(tw, lane * 8 * K + 4 * K, hi);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        sts[q] = lo[q];
-                        sts[4 + q] = hi[q];
-                    }
-                }
-                uint32_t out[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    __half2 h2 = __halves2half2(codebook_weight(sts[2 * q]), codebook_weight(sts[2 * q + 1]));
-                    out[q] = *reinterpret_cast<uint32_t *>(&h2);
-                }
-                // run (row u/2, half u%2) -> k row, first output channel of the 8
-                const int kr = trow * 16 + (lane >> 1);
-                const int n0 = tcol * 16 + (lane & 1) * 8;
-                unsigned char *dst = bt + ((n0 >> 6) * (kBK / 8) + (kr >> 3)) * 1024 + (kr & 7) * 128 +
-                                     ((((n0 & 63) >> 3) ^ (kr & 7)) << 4);
-                *reinterpret_cast<uint4 *>(dst) = make_uint4(out[0], out[1], out[2], out[3]);
+            // 4 tiles per warp; lane l decodes rows 2(l%8) and 2(l%8)+1 of tile
+            // l/8 (one parity per pass: compile-time bit windows)
+            static_assert((kBK / 16) * (kBN / 16) == 4 * kDecWarps, "tiles per stage");
+            {
+                const int T = dw * 4 + (lane >> 3);
+                const int trow = T / (kBN / 16), tcol = T - (T / (kBN / 16)) * (kBN / 16);
+                const uint32_t *tw = reinterpret_cast<const uint32_t *>(tr + T * 32 * K);
+                const int r0 = 2 * (lane & 7);
+                decode_row_to_b<K, 0>(tw, r0, p.cb, bt, trow, tcol);
+                decode_row_to_b<K, 1>(tw, r0 + 1, p.cb, bt, trow, tcol);
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -500,7 +507,8 @@ static exl3_status launch_gemm_t(const GemmParams &p, cudaStream_t stream)
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return EXL3_ERR_CUDA;
     const int tiles = ((p.m + kBM * kMT - 1) / (kBM * kMT)) * (p.n / kBN);
-    kern<<<tiles, kGemmThreads, smem, stream>>>(p);
+    if (launch_kernel(kern, dim3(tiles), dim3(kGemmThreads), (size_t)smem, stream, p) != cudaSuccess)
+        return EXL3_ERR_CUDA;
     return launch_status();
 }
 
@@ -532,9 +540,9 @@ extern "C" exl3_status exl3_gemm(const void *x, const uint16_t *trellis, const v
     int64_t rot_grid = (m * (k / 128) + 7) / 8;
     if (rot_grid > 148 * 16)
         rot_grid = 148 * 16;
-    rotate_tiled_kernel<<<(unsigned)rot_grid, 256, 0, s>>>((const __half *)x, (const __half *)suh, xt, (int)m,
-                                                           (int)k);
-    if (launch_status() != EXL3_OK)
+    if (launch_kernel(rotate_tiled_kernel, dim3((unsigned)rot_grid), dim3(256), 0, s, (const __half *)x,
+                      (const __half *)suh, xt, (int)m, (int)k) != cudaSuccess ||
+        launch_status() != EXL3_OK)
         return EXL3_ERR_CUDA;
     GemmParams p;
     p.xt = xt;
@@ -546,6 +554,7 @@ extern "C" exl3_status exl3_gemm(const void *x, const uint16_t *trellis, const v
     p.n = (int)n;
     p.status = (uint32_t *)ws;
     p.wait_ns = wait_limit_ns();
+    p.cb = codebook_constants();
     switch (K) {
     case 1: return launch_gemm_t<1>(p, s);
     case 2: return launch_gemm_t<2>(p, s);

@@ -4,34 +4,37 @@
 // bandwidth, so a dedicated GEMV path streams the quantised weights once).
 //
 // B200 design (the pages' consumer-GPU GEMV is prior art, not copied):
-//   * grid = (n/128 column blocks) x (k splits); one CTA = 1 producer warp +
-//     8 consumer warps, all on the same 128 output columns.
-//   * The producer warp streams the CTA's tile rows (8 tiles = 128 columns x
-//     16 input channels, 2K*128 bytes, contiguous in the trellis) into a ring
-//     of shared-memory stages with cp.async.bulk (no multicast), signalled on
-//     mbarriers; consumers release stages on a second set of mbarriers.  All
-//     waits are bounded (timeout -> status word, early exit).
-//   * Consumer warp w takes tile row w of every stage.  Lane (g, t) decodes,
-//     for each of 4 row groups q and 2 column halves, the run of 8
-//     consecutive weights of tile row 4q+t, columns 8(g&1).. of tile
-//     (4*half + g/2): one 64-bit read of the bit string, 8 windows, 8
-//     codebook words -- everything stays in registers.
-//   * The MAC runs on the tensor cores (mma.sync m16n8k16, fp32 accumulate).
-//     A codebook word's two fp16 halves are placed as a pair of k slots in B
-//     and the activation is duplicated across that pair in A, so the tensor
-//     core forms x*(hi + lo) exactly in fp32; the fp16 rounding of hi + lo
-//     that defines W_hat is skipped (the difference is at most half an fp16
-//     ulp of each weight, far inside the output tolerance).  The 8 weights of
-//     a run go to 4 MMAs (2 per MMA: k-pairs t and t+4 of output column
-//     parity 0 and 1); A rows are (batch, column parity) and zero elsewhere,
-//     so column parity never mixes.  Batch rows 0..7 per group, 2 groups for
-//     m > 8.
+//   * grid = (n/128 column blocks) x (k splits), 8 warps per CTA, all on the
+//     same 128 output columns (8 trellis tiles); warp w takes tile rows
+//     w, w+8, ... of the CTA's k range.  The split count is chosen so the
+//     CTAs fill whole waves of the GPU.
+//   * Lane (g, t) owns tile g of the column block and, in each of 4 row
+//     groups q, the whole tile row rho(q, t) (16 weights): rows are ordered
+//     so that all lanes of a group share the row parity, which makes every
+//     bit-window operation a compile-time byte permute (see row_states).
+//     Loads go straight from HBM into registers in this fragment order
+//     (read-only path, 8/16-byte vectors where aligned), one tile row ahead
+//     of the math -- no shared-memory staging, no bank conflicts.
+//   * The MAC runs on the tensor cores (mma.sync m16n8k16, fp32 accumulate):
+//     a codebook word's two fp16 halves form a pair of k slots in B and the
+//     activation is duplicated over that pair in A, so the tensor core forms
+//     x*(hi + lo) exactly in fp32 (the fp16 rounding of hi + lo that defines
+//     W_hat is skipped: at most half an fp16 ulp per weight, far inside the
+//     output tolerance).  Weights 2j, 2j+1 of a lane's row feed MMA j (k
+//     pairs t and t+4); A rows are (batch, column parity) with zeros
+//     elsewhere, so parities never mix.  The activation fragments are kept in
+//     shared memory as {x, 0, 0, x} records: one 8-byte load gives a lane its
+//     (a0, a2) pair for either parity.  Batch rows 0..7 per group, two groups
+//     for m > 8 (one decode feeds both).
 //   * x' = H(x .* suh)/sqrt(128) for the CTA's k range is computed once into
-//     shared memory (fp32 butterflies, rounded to fp16, stored duplicated).
+//     those records (fp32 butterflies, rounded to fp16).
 //   * Split-k: every CTA writes fp32 partials; the last CTA to arrive on the
 //     column block's counter (atomic ticket, no spinning) sums them in split
 //     order (deterministic), applies H/sqrt(128) and svh, writes fp16 y and
-//     re-arms the counter.
+//     re-arms the counter.  Nothing in the kernel waits on another CTA.
+//   * With EXL3_LAUNCH_PDL the first tile rows are requested before the
+//     kernel waits for its predecessor (griddepcontrol), and the next kernel
+//     is released as soon as this CTA's weight stream is consumed.
 #include <cuda_fp16.h>
 
 #include "exl3_device.cuh"
@@ -39,10 +42,8 @@
 
 namespace exl3 {
 
-constexpr int kGemvWarpsK = 8;        // consumer warps per CTA (one tile row each per stage)
-constexpr int kGemvThreads = 32 * (kGemvWarpsK + 1);
-constexpr int kGemvStages = 4;
-constexpr int kGemvRowsPerStage = kGemvWarpsK;  // tile rows per stage
+constexpr int kGemvWarps = 8;
+constexpr int kGemvThreads = 32 * kGemvWarps;
 
 struct GemvParams {
     const __half *x;
@@ -52,123 +53,152 @@ struct GemvParams {
     __half *y;
     int m, k, n;
     int splits;
-    int rows_per_split;  // tile rows (of 16 input channels) per split, last may be shorter
+    int rows_per_split;  // tile rows (16 input channels each) per split; last may be shorter
     float *partials;     // [splits][m][n]
     uint32_t *counters;  // [n / 128]
-    uint32_t *status;
-    uint64_t wait_ns;    // bound of every device wait
+    Codebook cb;
 };
 
-// Shared memory carve-up (bytes), all 16-byte aligned.
-struct GemvSmem {
-    int bars;      // 2 * stages mbarriers
-    int flag;      // last-CTA flag
-    int xs;        // dup'd x' [k_local][m] u32
-    int stage;     // stages of tile rows
-    int red;       // [warps][m][128] f32 reduction buffer (aliases stages)
-    int total;
+// Activation records, in MMA A-fragment register order.  For batch group mg
+// (batches 8mg..8mg+7), quad ba (batches 8mg+ba and 8mg+ba+4) and A-row
+// parity p, a 16-byte record holds the lane's {a0, a1, a2, a3}:
+//   p = 0: {x(8mg+ba), x(8mg+ba+4), 0, 0}     p = 1: {0, 0, x(8mg+ba), x(8mg+ba+4)}
+// with x the rotated activation duplicated in both fp16 halves (absent batches
+// are zero).  Only quads holding a batch < m are stored; per input channel
+// there are rec_slots(m) records.
+__host__ __device__ inline int rec_quads(int m, int mg)
+{
+    const int q = m - 8 * mg;
+    return q <= 0 ? 0 : (q < 4 ? q : 4);
+}
+
+__host__ __device__ inline int rec_slots(int m)
+{
+    return 2 * (rec_quads(m, 0) + rec_quads(m, 1));
+}
+
+// Dynamic shared memory: a flag, one zero record, then the records
+// [k_local][rec_slots] (16 B each), later reused as the cross-warp reduction
+// buffer [warps][m][128] f32.
+__host__ __device__ inline int gemv_smem_bytes(int m, int rows_per_split)
+{
+    const int rec = rows_per_split * 16 * rec_slots(m) * 16;
+    const int red = kGemvWarps * m * 128 * 4;
+    return 32 + (rec > red ? rec : red);
+}
+
+// Row of tile-row group q for lane t: groups 0,1 take the even rows, groups
+// 2,3 the odd rows, so a group's lanes share the row parity.
+__device__ __forceinline__ int row_of(int q, int t)
+{
+    return 2 * (4 * (q & 1) + t) + (q >> 1);
+}
+
+template <int K>
+struct RowBuf {
+    static constexpr int N =
+        RowSpan<K, 0>::N32 > RowSpan<K, 1>::N32 ? RowSpan<K, 0>::N32 : RowSpan<K, 1>::N32;
+    uint32_t w[4][N];
 };
 
 template <int K>
-__host__ __device__ constexpr int gemv_stage_bytes()
+__device__ __forceinline__ void load_tile_row(const uint32_t *tile, int t, RowBuf<K> &b)
 {
-    return kGemvRowsPerStage * 8 * 32 * K;  // 8 tiles of 32K bytes per tile row
+    load_row<K, 0>(tile, row_of(0, t), b.w[0]);
+    load_row<K, 0>(tile, row_of(1, t), b.w[1]);
+    load_row<K, 1>(tile, row_of(2, t), b.w[2]);
+    load_row<K, 1>(tile, row_of(3, t), b.w[3]);
 }
 
-__host__ __device__ inline GemvSmem gemv_smem_layout(int K, int m, int rows_per_split)
+// Activation-record address of one lane for one batch group (zero record,
+// stride 0, when the lane's quad holds no batch).
+struct RecPtr {
+    const unsigned char *base;
+    int stride;
+};
+
+template <int K, int MG>
+__device__ __forceinline__ void mac_tile_row(const RowBuf<K> &buf, int kl0, const RecPtr (&rp)[MG], int t,
+                                             const Codebook &cb, float (&acc)[MG][8][4])
 {
-    GemvSmem s;
-    s.bars = 0;
-    s.flag = 2 * kGemvStages * 8;
-    s.xs = (s.flag + 16 + 15) & ~15;
-    const int xs_bytes = rows_per_split * 16 * m * 4;
-    s.stage = (s.xs + xs_bytes + 127) & ~127;
-    const int stage_bytes = kGemvRowsPerStage * 8 * 32 * K;
-    const int red_bytes = kGemvWarpsK * m * 128 * 4;
-    s.red = s.stage;
-    const int body = kGemvStages * stage_bytes > red_bytes ? kGemvStages * stage_bytes : red_bytes;
-    s.total = s.stage + body;
-    return s;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int kl = kl0 + row_of(q, t);
+        uint32_t A[MG][4];
+#pragma unroll
+        for (int mg = 0; mg < MG; ++mg) {
+            const uint4 r = *reinterpret_cast<const uint4 *>(rp[mg].base + kl * rp[mg].stride);
+            A[mg][0] = r.x;
+            A[mg][1] = r.y;
+            A[mg][2] = r.z;
+            A[mg][3] = r.w;
+        }
+        uint32_t s[16];
+        if (q < 2)
+            row_states<K, RowSpan<K, 0>::P>(buf.w[q], s);
+        else
+            row_states<K, RowSpan<K, 1>::P>(buf.w[q], s);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const uint32_t b0 = codebook_word(s[2 * j], cb);
+            const uint32_t b1 = codebook_word(s[2 * j + 1], cb);
+#pragma unroll
+            for (int mg = 0; mg < MG; ++mg)
+                mma_16816(acc[mg][j], A[mg], b0, b1);
+        }
+    }
 }
 
 template <int K, int MG>
-__global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvParams p)
+__global__ void __launch_bounds__(kGemvThreads, MG == 1 ? 2 : 1) gemv_kernel(const GemvParams p)
 {
-    extern __shared__ __align__(128) unsigned char smem[];
-    const GemvSmem L = gemv_smem_layout(K, p.m, p.rows_per_split);
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bars);
-    uint64_t *empty = full + kGemvStages;
-    volatile int *flag = reinterpret_cast<volatile int *>(smem + L.flag);
-    uint32_t *xs = reinterpret_cast<uint32_t *>(smem + L.xs);
-    unsigned char *stage_base = smem + L.stage;
+    extern __shared__ __align__(16) unsigned char smem[];
+    volatile int *flag = reinterpret_cast<volatile int *>(smem);
+    unsigned char *zero_rec = smem + 16;  // 16 zero bytes
+    unsigned char *recs = smem + 32;      // x' records, later the reduction buffer
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
     const int nb = blockIdx.x, split = blockIdx.y;
     const int m = p.m, n = p.n;
     const int tn_count = n >> 4;
     const int row_begin = split * p.rows_per_split;
     int row_end = row_begin + p.rows_per_split;
-    const int tr_total = p.k >> 4;
-    if (row_end > tr_total)
-        row_end = tr_total;
+    if (row_end > (p.k >> 4))
+        row_end = p.k >> 4;
     const int rows = row_end - row_begin;
-    const int n_stage_iters = (rows + kGemvRowsPerStage - 1) / kGemvRowsPerStage;
-    constexpr int kStageBytes = gemv_stage_bytes<K>();
-    constexpr int kRowBytes = 8 * 32 * K;  // one tile row of 8 tiles
 
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < kGemvStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kGemvWarpsK);
-        }
-        *flag = 0;
-        fence_mbar_init();
+    // this warp's first two tile rows: requested before anything else
+    const uint32_t *tiles =
+        reinterpret_cast<const uint32_t *>(p.trellis) + ((int64_t)nb * 8 + g) * 8 * K;
+    const int64_t row_stride = (int64_t)tn_count * 8 * K;  // u32 per tile row of the matrix
+    RowBuf<K> buf0, buf1, buf2;
+    int tr = warp;
+    if (tr < rows)
+        load_tile_row<K>(tiles + (int64_t)(row_begin + tr) * row_stride, t, buf0);
+    if (tr + kGemvWarps < rows)
+        load_tile_row<K>(tiles + (int64_t)(row_begin + tr + kGemvWarps) * row_stride, t, buf1);
+    const Codebook cb = p.cb;
+
+    // everything below reads x or touches the workspace/output: wait for the
+    // preceding kernel (a no-op unless launched with programmatic overlap)
+    grid_dep_wait();
+
+    // activation records for this split's k range: zero, then fill
+    const int slots = rec_slots(m);
+    {
+        uint4 *r4 = reinterpret_cast<uint4 *>(smem + 16);  // zero record + records
+        const int n4 = 1 + rows * 16 * slots;
+        for (int i = threadIdx.x; i < n4; i += kGemvThreads)
+            r4[i] = make_uint4(0u, 0u, 0u, 0u);
     }
     __syncthreads();
-
-    if (warp == kGemvWarpsK) {
-        // ------------------------------------------------------ producer ---
-        if (lane == 0) {
-            bool ok = true;
-            int issued = 0;
-            for (int it = 0; it < n_stage_iters; ++it) {
-                const int s = it % kGemvStages;
-                const uint32_t ph = (uint32_t)(it / kGemvStages) & 1u;
-                if (!mbar_wait(&empty[s], ph ^ 1u, p.wait_ns)) {
-                    ok = false;
-                    break;
-                }
-                const int r0 = row_begin + it * kGemvRowsPerStage;
-                int nr = row_end - r0;
-                if (nr > kGemvRowsPerStage)
-                    nr = kGemvRowsPerStage;
-                mbar_arrive_expect_tx(&full[s], (uint32_t)(nr * kRowBytes));
-                for (int r = 0; r < nr; ++r) {
-                    const uint16_t *src =
-                        p.trellis + ((int64_t)(r0 + r) * tn_count + (int64_t)nb * 8) * 16 * K;
-                    bulk_g2s(stage_base + s * kStageBytes + r * kRowBytes, src, kRowBytes, &full[s]);
-                }
-                issued = it + 1;
-            }
-            if (!ok)
-                record_timeout(p.status);
-            // never leave while copies into this CTA's shared memory are in flight
-            for (int it = (issued > kGemvStages ? issued - kGemvStages : 0); it < issued; ++it) {
-                const int s = it % kGemvStages;
-                if (!mbar_wait(&full[s], (uint32_t)(it / kGemvStages) & 1u, kDefaultWaitNs))
-                    record_timeout(p.status);
-            }
-        }
-        return;
-    }
-
-    // ----------------------------------------------------------- consumers ---
-    // x' for this split's k range: warp w rotates 128-channel blocks w, w+8, ...
     {
         const int k0 = row_begin * 16;
-        const int nblk = rows * 16 / 128;
-        for (int job = warp; job < nblk * m; job += kGemvWarpsK) {
-            const int b = job / nblk, blk = job - (job / nblk) * nblk;
+        const int nblk = rows / 8;
+        const int q0 = rec_quads(m, 0);
+        for (int job = warp; job < nblk * m; job += kGemvWarps) {
+            const int b = job / nblk, blk = job - b * nblk;
             const int c = k0 + blk * 128 + lane * 4;
             const uint2 raw = *reinterpret_cast<const uint2 *>(p.x + (int64_t)b * p.k + c);
             const uint2 sr = *reinterpret_cast<const uint2 *>(p.suh + c);
@@ -177,142 +207,111 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvParams p)
             float v[4] = {__low2float(xv[0]) * __low2float(sv[0]), __high2float(xv[0]) * __high2float(sv[0]),
                           __low2float(xv[1]) * __low2float(sv[1]), __high2float(xv[1]) * __high2float(sv[1])};
             warp_fwht128(v);
+            const int mg = b >> 3, bb = b & 7, ba = bb & 3, hi = bb >> 2;
+            const int slot = 2 * (mg * q0 + ba);  // the even-parity record; +1 is the odd one
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const __half h = __float2half_rn(v[e] * 0.08838834764831845f);
-                const uint32_t hb = (uint32_t)__half_as_ushort(h);
-                xs[(blk * 128 + lane * 4 + e) * m + b] = hb | (hb << 16);
+                const uint32_t h = (uint32_t)__half_as_ushort(__float2half_rn(v[e] * 0.08838834764831845f));
+                uint32_t *rec = reinterpret_cast<uint32_t *>(recs + ((blk * 128 + lane * 4 + e) * slots + slot) * 16);
+                rec[hi] = h | (h << 16);      // even record: field 0 (batch ba) or 1 (ba + 4)
+                rec[4 + 2 + hi] = h | (h << 16);  // odd record: field 2 or 3
             }
         }
     }
-    asm volatile("bar.sync 1, %0;\n" ::"r"(32 * kGemvWarpsK));
+    __syncthreads();
 
-    const int g = lane >> 2, t = lane & 3;
-    const bool odd = (g & 1) != 0;
-    float acc[MG][2][4][4];
+    RecPtr rp[MG];
+#pragma unroll
+    for (int mg = 0; mg < MG; ++mg) {
+        const int ba = g >> 1;
+        const int qbase = mg * rec_quads(m, 0);
+        if (ba < rec_quads(m, mg)) {
+            rp[mg].base = recs + (2 * (qbase + ba) + (g & 1)) * 16;
+            rp[mg].stride = slots * 16;
+        } else {
+            rp[mg].base = zero_rec;
+            rp[mg].stride = 0;
+        }
+    }
+
+    float acc[MG][8][4];
 #pragma unroll
     for (int a = 0; a < MG; ++a)
 #pragma unroll
-        for (int b = 0; b < 2; ++b)
+        for (int j = 0; j < 8; ++j)
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
-#pragma unroll
-                for (int d = 0; d < 4; ++d)
-                    acc[a][b][c][d] = 0.f;
+            for (int e = 0; e < 4; ++e)
+                acc[a][j][e] = 0.f;
 
-    bool ok = true;
-    for (int it = 0; it < n_stage_iters; ++it) {
-        const int s = it % kGemvStages;
-        if (!warp_wait(&full[s], (uint32_t)(it / kGemvStages) & 1u, p.wait_ns)) {
-            ok = false;
+    // three buffers in rotation: two tile rows' loads are in flight during the math
+    constexpr int W = kGemvWarps;
+    for (; tr < rows;) {
+        if (tr + 2 * W < rows)
+            load_tile_row<K>(tiles + (int64_t)(row_begin + tr + 2 * W) * row_stride, t, buf2);
+        mac_tile_row<K, MG>(buf0, tr * 16, rp, t, cb, acc);
+        tr += W;
+        if (tr >= rows)
             break;
-        }
-        const int rl = it * kGemvRowsPerStage + warp;  // local tile row of this warp
-        if (rl < rows) {
-            const uint32_t *row_tiles =
-                reinterpret_cast<const uint32_t *>(stage_base + s * kStageBytes + warp * kRowBytes);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int kl = rl * 16 + 4 * q + t;
-                uint32_t A[MG][4];
-#pragma unroll
-                for (int mg = 0; mg < MG; ++mg) {
-                    const int ba = 8 * mg + (g >> 1), bb = ba + 4;
-                    const uint32_t xa = ba < m ? xs[kl * m + ba] : 0u;
-                    const uint32_t xb = bb < m ? xs[kl * m + bb] : 0u;
-                    A[mg][0] = odd ? 0u : xa;
-                    A[mg][1] = odd ? 0u : xb;
-                    A[mg][2] = odd ? xa : 0u;
-                    A[mg][3] = odd ? xb : 0u;
-                }
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const uint32_t *tile = row_tiles + (4 * h + (g >> 1)) * 8 * K;
-                    const int start = (16 * (4 * q + t) + 8 * (g & 1)) * K;
-                    uint32_t st[8];
-                    if constexpr (K <= 6) {
-                        run_states<K, 8>(tile, start, st);
-                    } else {
-                        uint32_t lo[4], hi[4];
-                        run_states<K, 4>(tile, start, lo);
-                        run_states<K, 4>(tile, start + 4 * K, hi);
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            st[j] = lo[j];
-                            st[4 + j] = hi[j];
-                        }
-                    }
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const uint32_t b0 = codebook_word(st[2 * j]);
-                        const uint32_t b1 = codebook_word(st[2 * j + 1]);
-#pragma unroll
-                        for (int mg = 0; mg < MG; ++mg)
-                            mma_16816(acc[mg][h][j], A[mg], b0, b1);
-                    }
-                }
-            }
-        }
-        __syncwarp();
-        if (lane == 0)
-            mbar_arrive(&empty[s]);
+        if (tr + 2 * W < rows)
+            load_tile_row<K>(tiles + (int64_t)(row_begin + tr + 2 * W) * row_stride, t, buf0);
+        mac_tile_row<K, MG>(buf1, tr * 16, rp, t, cb, acc);
+        tr += W;
+        if (tr >= rows)
+            break;
+        if (tr + 2 * W < rows)
+            load_tile_row<K>(tiles + (int64_t)(row_begin + tr + 2 * W) * row_stride, t, buf1);
+        mac_tile_row<K, MG>(buf2, tr * 16, rp, t, cb, acc);
+        tr += W;
     }
-    if (!ok) {
-        record_timeout(p.status);
-        *flag = -1;
-    }
+
+    // the weight stream of this CTA is done: let the next kernel start launching
+    grid_dep_launch();
 
     // ------------------------------------------------- reduce across warps ---
-    asm volatile("bar.sync 1, %0;\n" ::"r"(32 * kGemvWarpsK));
-    float *red = reinterpret_cast<float *>(smem + L.red);  // [warp][m][128]
-    // accumulator element (mg, h, j, e): row i = g (+8 for e >= 2) -> batch
-    // 8mg + i/2, column parity i&1; n-slot 2t (+1 for odd e) -> column group
-    // 64h + 8*slot, column within group 2j + parity.
+    __syncthreads();  // records no longer needed: reuse as [warp][m][128] f32
+    float *red = reinterpret_cast<float *>(recs);
+    // accumulator (mg, j, e): A row i = g (+8 for e >= 2) -> batch 8mg + i/2,
+    // column parity i&1; n-slot 2t (+1 for odd e) -> tile of the block;
+    // column = 16 * slot + 2j + parity.
 #pragma unroll
     for (int mg = 0; mg < MG; ++mg)
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
+        for (int j = 0; j < 8; ++j)
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int i = g + ((e >> 1) << 3);
-                    const int b = 8 * mg + (i >> 1);
-                    const int slot = 2 * t + (e & 1);
-                    const int col = 64 * h + 8 * slot + 2 * j + (i & 1);
-                    if (b < m)
-                        red[(warp * m + b) * 128 + col] = acc[mg][h][j][e];
-                }
-    asm volatile("bar.sync 1, %0;\n" ::"r"(32 * kGemvWarpsK));
-    if (*flag < 0)
-        return;
-    const int tid = threadIdx.x;  // 0 .. 255 among consumers
-    for (int e = tid; e < m * 128; e += 32 * kGemvWarpsK) {
+            for (int e = 0; e < 4; ++e) {
+                const int i = g + ((e >> 1) << 3);
+                const int b = 8 * mg + (i >> 1);
+                const int col = 16 * (2 * t + (e & 1)) + 2 * j + (i & 1);
+                if (b < m)
+                    red[(warp * m + b) * 128 + col] = acc[mg][j][e];
+            }
+    __syncthreads();
+    const int tid = threadIdx.x;
+    for (int e = tid; e < m * 128; e += kGemvThreads) {
         float sum = 0.f;
 #pragma unroll
-        for (int w = 0; w < kGemvWarpsK; ++w)
+        for (int w = 0; w < kGemvWarps; ++w)
             sum += red[w * m * 128 + e];
-        red[e] = sum;  // row 0 of the buffer now holds the CTA's partial; w = 0 is read first
+        red[e] = sum;
     }
-    asm volatile("bar.sync 1, %0;\n" ::"r"(32 * kGemvWarpsK));
+    __syncthreads();
 
     if (p.splits > 1) {
-        // publish partial, take a ticket; the last CTA finishes the block
-        for (int e = tid; e < m * 128; e += 32 * kGemvWarpsK) {
+        for (int e = tid; e < m * 128; e += kGemvThreads) {
             const int b = e >> 7, c = e & 127;
             p.partials[((int64_t)split * m + b) * n + nb * 128 + c] = red[e];
         }
         __threadfence();
-        asm volatile("bar.sync 1, %0;\n" ::"r"(32 * kGemvWarpsK));
+        __syncthreads();
         if (tid == 0) {
             const uint32_t ticket = atomicAdd(&p.counters[nb], 1u);
             *flag = (ticket == (uint32_t)(p.splits - 1)) ? 1 : 0;
         }
-        asm volatile("bar.sync 1, %0;\n" ::"r"(32 * kGemvWarpsK));
+        __syncthreads();
         if (*flag != 1)
             return;
         __threadfence();
-        for (int e = tid; e < m * 128; e += 32 * kGemvWarpsK) {
+        for (int e = tid; e < m * 128; e += kGemvThreads) {
             const int b = e >> 7, c = e & 127;
             float sum = 0.f;
             for (int sp = 0; sp < p.splits; ++sp)
@@ -321,11 +320,11 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvParams p)
         }
         if (tid == 0)
             p.counters[nb] = 0u;
-        asm volatile("bar.sync 1, %0;\n" ::"r"(32 * kGemvWarpsK));
+        __syncthreads();
     }
 
     // ------------------------------------ output rotation, scales, fp16 y ---
-    for (int b = warp; b < m; b += kGemvWarpsK) {
+    for (int b = warp; b < m; b += kGemvWarps) {
         float v[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e)
@@ -352,50 +351,59 @@ struct GemvPlan {
 
 static int g_num_sms = 0;
 
-static int num_sms()
+int num_sms()
 {
     if (g_num_sms <= 0) {
         int dev = 0;
-        cudaGetDevice(&dev);
         int v = 0;
-        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) {
+            cudaGetLastError();
             v = 148;
+        }
         g_num_sms = v;
     }
     return g_num_sms;
 }
 
-// Splits so that about two CTAs per SM are in flight; each split covers a
-// whole number of 128-channel blocks (8 tile rows) and its rotated
-// activations fit in 64 KB of shared memory.
-static GemvPlan gemv_plan(int64_t m, int64_t k, int64_t n, int K, int sms)
+// Split count: each split covers whole 128-channel blocks and its x' records
+// fit 96 KB of shared memory (192 KB for m > 8, one CTA per SM); among the candidates take the smallest
+// estimated time = waves x (blocks per split + 1), a wave being the resident
+// CTAs (2 per SM for m <= 8, 1 above) and the +1 the per-CTA fixed cost; ties go to fewer splits.
+static GemvPlan gemv_plan(int64_t m, int64_t k, int64_t n, int sms)
 {
     GemvPlan pl;
     const int64_t blocks_k = k / 128;
     const int64_t nblocks = n / 128;
-    int64_t splits = (2 * sms + nblocks - 1) / nblocks;
-    if (splits > blocks_k)
-        splits = blocks_k;
-    if (splits < 1)
-        splits = 1;
-    // shared-memory cap on the rotated activations: rows*16*m*4 <= 64 KB
-    const int64_t max_blocks = (64 * 1024) / (128 * m * 4);
-    int64_t per = (blocks_k + splits - 1) / splits;
-    if (per > max_blocks)
-        per = max_blocks;
-    if (per < 1)
-        per = 1;
-    splits = (blocks_k + per - 1) / per;
-    pl.splits = (int)splits;
-    pl.rows_per_split = (int)(per * 8);
-    pl.smem = gemv_smem_layout(K, (int)m, pl.rows_per_split).total;
+    const int64_t slots = (m <= 8 ? 2 : 1) * (int64_t)sms;  // resident CTAs per SM
+    const int64_t rec_budget = (m <= 8 ? 96 : 192) * 1024;  // x' records per CTA
+    int64_t max_per = rec_budget / (128 * rec_slots((int)m) * 16);
+    if (max_per < 1)
+        max_per = 1;
+    int64_t best_per = blocks_k < max_per ? blocks_k : max_per, best_cost = -1;
+    for (int64_t s = 1; s <= blocks_k && s <= 64; ++s) {
+        const int64_t per = (blocks_k + s - 1) / s;
+        if (per > max_per)
+            continue;
+        const int64_t real_s = (blocks_k + per - 1) / per;
+        const int64_t units = nblocks * real_s;
+        const int64_t waves = (units + slots - 1) / slots;
+        const int64_t cost = waves * (per + 1) * 64 + real_s;
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best_per = per;
+        }
+    }
+    pl.splits = (int)((blocks_k + best_per - 1) / best_per);
+    pl.rows_per_split = (int)(best_per * 8);
+    pl.smem = gemv_smem_bytes((int)m, pl.rows_per_split);
     return pl;
 }
 
-size_t gemv_workspace_bytes(int64_t m, int64_t k, int64_t n, int K, int sms)
+size_t gemv_workspace_bytes(int64_t m, int64_t k, int64_t n, int sms)
 {
-    const GemvPlan pl = gemv_plan(m, k, n, K, sms);
-    size_t bytes = 256;                                // status word + padding
+    const GemvPlan pl = gemv_plan(m, k, n, sms);
+    size_t bytes = 256;                                  // status word + padding
     bytes += (size_t)((n / 128) * 4 + 255) / 256 * 256;  // counters
     if (pl.splits > 1)
         bytes += (size_t)pl.splits * (size_t)m * (size_t)n * 4;
@@ -406,10 +414,12 @@ template <int K, int MG>
 static exl3_status launch_gemv_t(const GemvParams &p, int smem, cudaStream_t stream)
 {
     auto kern = gemv_kernel<K, MG>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return EXL3_ERR_CUDA;
     dim3 grid((unsigned)(p.n / 128), (unsigned)p.splits);
-    kern<<<grid, kGemvThreads, smem, stream>>>(p);
+    if (launch_kernel(kern, grid, dim3(kGemvThreads), (size_t)smem, stream, p) != cudaSuccess)
+        return EXL3_ERR_CUDA;
     return launch_status();
 }
 
@@ -433,8 +443,8 @@ exl3_status run_gemv(const void *x, const uint16_t *trellis, const void *suh, co
                      size_t workspace_bytes, cudaStream_t stream)
 {
     const int sms = num_sms();
-    const GemvPlan pl = gemv_plan(m, k, n, K, sms);
-    if (!workspace || !aligned16(workspace) || workspace_bytes < gemv_workspace_bytes(m, k, n, K, sms))
+    const GemvPlan pl = gemv_plan(m, k, n, sms);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < gemv_workspace_bytes(m, k, n, sms))
         return EXL3_ERR_WORKSPACE;
     unsigned char *ws = (unsigned char *)workspace;
     GemvParams p;
@@ -448,10 +458,9 @@ exl3_status run_gemv(const void *x, const uint16_t *trellis, const void *suh, co
     p.n = (int)n;
     p.splits = pl.splits;
     p.rows_per_split = pl.rows_per_split;
-    p.status = (uint32_t *)ws;
     p.counters = (uint32_t *)(ws + 256);
     p.partials = (float *)(ws + 256 + (size_t)((n / 128) * 4 + 255) / 256 * 256);
-    p.wait_ns = wait_limit_ns();
+    p.cb = codebook_constants();
     if (m <= 8)
         return launch_gemv_k<1>(p, K, pl.smem, stream);
     return launch_gemv_k<2>(p, K, pl.smem, stream);
@@ -463,7 +472,7 @@ extern "C" size_t exl3_gemv_workspace_size(int64_t m, int64_t k, int64_t n, int 
 {
     if (m < 1 || m > 16 || k < 128 || n < 128 || (k % 128) || (n % 128) || K < 1 || K > 8)
         return 0;
-    return exl3::gemv_workspace_bytes(m, k, n, K, exl3::num_sms());
+    return exl3::gemv_workspace_bytes(m, k, n, exl3::num_sms());
 }
 
 extern "C" exl3_status exl3_gemv(const void *x, const uint16_t *trellis, const void *suh,

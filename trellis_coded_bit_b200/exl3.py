@@ -23,7 +23,10 @@ EXL3_ERR_TIMEOUT = 5
 # Every symbol the public headers declare.
 EXPORTED = ["exl3_status_string", "exl3_version", "exl3_hadamard", "exl3_decode_tiles",
             "exl3_gemv_workspace_size", "exl3_gemv", "exl3_gemm_workspace_size", "exl3_gemm",
-            "exl3_workspace_status", "exl3_debug_set_wait_limit_ns", "exl3_debug_wait_limit_ns"]
+            "exl3_workspace_status", "exl3_set_launch_flags", "exl3_launch_flags",
+            "exl3_debug_set_wait_limit_ns", "exl3_debug_wait_limit_ns"]
+
+EXL3_LAUNCH_PDL = 1
 
 _lib = None
 _lock = threading.Lock()
@@ -67,6 +70,10 @@ def load(build_if_needed=True):
             getattr(lib, name).restype = ci
         lib.exl3_workspace_status.argtypes = [vp, sz, ci, vp]
         lib.exl3_workspace_status.restype = ci
+        lib.exl3_set_launch_flags.argtypes = [ctypes.c_uint]
+        lib.exl3_set_launch_flags.restype = None
+        lib.exl3_launch_flags.argtypes = []
+        lib.exl3_launch_flags.restype = ctypes.c_uint
         lib.exl3_debug_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         lib.exl3_debug_set_wait_limit_ns.restype = None
         lib.exl3_debug_wait_limit_ns.argtypes = []
@@ -172,6 +179,15 @@ def exl3_workspace_status(workspace, clear=False, stream=None):
     """Status word of a gemv/gemm workspace (synchronises the stream)."""
     return int(load().exl3_workspace_status(_dev(workspace, torch.uint8, "workspace"), workspace.numel(),
                                             1 if clear else 0, _stream(stream)))
+
+
+def exl3_set_launch_flags(flags):
+    """EXL3_LAUNCH_PDL: programmatic dependent launch (weights must be immutable)."""
+    load().exl3_set_launch_flags(int(flags))
+
+
+def exl3_launch_flags():
+    return int(load().exl3_launch_flags())
 
 
 def exl3_debug_set_wait_limit_ns(ns):
