@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--no-gemm", action="store_true", help="skip the m=2048 GEMM line item")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-pdl", action="store_true",
+                    help="launch without programmatic dependent launch (PDL is valid here: weights are immutable)")
     return ap.parse_args()
 
 
@@ -197,6 +199,8 @@ def run_ours(args, rank, world, local_rank):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     exl3.load()
+    if not args.no_pdl:
+        exl3.exl3_set_launch_flags(exl3.EXL3_LAUNCH_PDL)
     peaks = load_peaks()
     layers = make_layers()
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
@@ -315,6 +319,7 @@ def run_ours(args, rank, world, local_rank):
                            "trellis_bytes_per_step": sum(L.trellis.nbytes for L in layers),
                            "l2": "inputs larger than L2 (398 MB of trellis rotated per step)",
                            "timing": "CUDA graph of one step, CUDA events on the launching stream",
+                           "launch": "programmatic dependent launch" if not args.no_pdl else "plain",
                            "parallelism": "replica per GPU" if world > 1 else "single GPU"},
                 "roofline": roof, "gpu_launches": len(D) * args.steps,
                 "e2e": {"value": step_bytes / (e2e_ms * 1e-3) / 1e9 * world, "unit": "GB/s",

@@ -200,6 +200,38 @@ def test_gemm_timeout_reports_status_without_hang():
     check_layer(layer, y)
 
 
+def test_pdl_launches_give_identical_results():
+    # a chain of dependent calls (each layer's input is the previous layer's output) run with
+    # and without programmatic dependent launch must agree bit for bit
+    layers = [inputs.make_layer(1, 1024, 1024, K, seed=40 + K) for K in (2, 3, 4)]
+    big = inputs.make_layer(256, 1024, 1024, 4, seed=44)
+    dl = [(dev(L.trellis), dev(L.suh), dev(L.svh), L.K) for L in layers]
+    db = (dev(big.trellis), dev(big.suh), dev(big.svh), big.K)
+    x0 = dev(layers[0].x)
+    xb = dev(big.x)
+    ws = exl3.new_workspace(max(exl3.exl3_gemv_workspace_size(1, 1024, 1024, 4),
+                                exl3.exl3_gemm_workspace_size(256, 1024, 1024, 4)))
+
+    def chain():
+        y = x0
+        for t, suh, svh, K in dl * 3:
+            y = exl3.exl3_gemv(y, t, suh, svh, K, workspace=ws)
+        z = xb
+        for _ in range(3):
+            z = exl3.exl3_gemm(z, db[0], db[1], db[2], db[3], workspace=ws)
+        torch.cuda.synchronize()
+        return y.cpu().numpy(), z.cpu().numpy()
+
+    ref = chain()
+    try:
+        exl3.exl3_set_launch_flags(exl3.EXL3_LAUNCH_PDL)
+        got = chain()
+    finally:
+        exl3.exl3_set_launch_flags(0)
+    assert np.array_equal(ref[0], got[0]) and np.array_equal(ref[1], got[1])
+    assert np.isfinite(ref[0]).all() and np.isfinite(ref[1]).all()
+
+
 def test_native_library_is_the_in_tree_build():
     import os
 

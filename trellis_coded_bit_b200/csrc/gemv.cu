@@ -184,39 +184,47 @@ __global__ void __launch_bounds__(kGemvThreads, MG == 1 ? 2 : 1) gemv_kernel(con
     // preceding kernel (a no-op unless launched with programmatic overlap)
     grid_dep_wait();
 
-    // activation records for this split's k range: zero, then fill
+    // activation records for this split's k range.  A job is (quad, 128-block):
+    // the warp rotates the quad's one or two batches and writes whole records
+    // (both parities), so no zero-fill pass is needed.
     const int slots = rec_slots(m);
-    {
-        uint4 *r4 = reinterpret_cast<uint4 *>(smem + 16);  // zero record + records
-        const int n4 = 1 + rows * 16 * slots;
-        for (int i = threadIdx.x; i < n4; i += kGemvThreads)
-            r4[i] = make_uint4(0u, 0u, 0u, 0u);
-    }
-    __syncthreads();
     {
         const int k0 = row_begin * 16;
         const int nblk = rows / 8;
-        const int q0 = rec_quads(m, 0);
-        for (int job = warp; job < nblk * m; job += kGemvWarps) {
-            const int b = job / nblk, blk = job - b * nblk;
+        const int q0 = rec_quads(m, 0), nq = q0 + rec_quads(m, 1);
+        const float s128 = 0.08838834764831845f;
+        for (int job = warp; job < nq * nblk; job += kGemvWarps) {
+            const int qd = job / nblk, blk = job - qd * nblk;
+            const int mg = qd >= q0 ? 1 : 0, ba = qd - mg * q0;
+            const int b0 = 8 * mg + ba, b1 = b0 + 4;
             const int c = k0 + blk * 128 + lane * 4;
-            const uint2 raw = *reinterpret_cast<const uint2 *>(p.x + (int64_t)b * p.k + c);
             const uint2 sr = *reinterpret_cast<const uint2 *>(p.suh + c);
-            const __half2 *xv = reinterpret_cast<const __half2 *>(&raw);
+            const uint2 r0 = *reinterpret_cast<const uint2 *>(p.x + (int64_t)b0 * p.k + c);
+            uint2 r1 = make_uint2(0u, 0u);
+            if (b1 < m)
+                r1 = *reinterpret_cast<const uint2 *>(p.x + (int64_t)b1 * p.k + c);
             const __half2 *sv = reinterpret_cast<const __half2 *>(&sr);
-            float v[4] = {__low2float(xv[0]) * __low2float(sv[0]), __high2float(xv[0]) * __high2float(sv[0]),
-                          __low2float(xv[1]) * __low2float(sv[1]), __high2float(xv[1]) * __high2float(sv[1])};
-            warp_fwht128(v);
-            const int mg = b >> 3, bb = b & 7, ba = bb & 3, hi = bb >> 2;
-            const int slot = 2 * (mg * q0 + ba);  // the even-parity record; +1 is the odd one
+            const __half2 *x0 = reinterpret_cast<const __half2 *>(&r0);
+            const __half2 *x1 = reinterpret_cast<const __half2 *>(&r1);
+            float v0[4] = {__low2float(x0[0]) * __low2float(sv[0]), __high2float(x0[0]) * __high2float(sv[0]),
+                           __low2float(x0[1]) * __low2float(sv[1]), __high2float(x0[1]) * __high2float(sv[1])};
+            float v1[4] = {__low2float(x1[0]) * __low2float(sv[0]), __high2float(x1[0]) * __high2float(sv[0]),
+                           __low2float(x1[1]) * __low2float(sv[1]), __high2float(x1[1]) * __high2float(sv[1])};
+            warp_fwht128(v0);
+            if (b1 < m)
+                warp_fwht128(v1);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const uint32_t h = (uint32_t)__half_as_ushort(__float2half_rn(v[e] * 0.08838834764831845f));
-                uint32_t *rec = reinterpret_cast<uint32_t *>(recs + ((blk * 128 + lane * 4 + e) * slots + slot) * 16);
-                rec[hi] = h | (h << 16);      // even record: field 0 (batch ba) or 1 (ba + 4)
-                rec[4 + 2 + hi] = h | (h << 16);  // odd record: field 2 or 3
+                const uint32_t h0 = (uint32_t)__half_as_ushort(__float2half_rn(v0[e] * s128));
+                const uint32_t h1 = b1 < m ? (uint32_t)__half_as_ushort(__float2half_rn(v1[e] * s128)) : 0u;
+                const uint32_t d0 = h0 | (h0 << 16), d1 = h1 | (h1 << 16);
+                uint4 *rec = reinterpret_cast<uint4 *>(recs + ((blk * 128 + lane * 4 + e) * slots + 2 * qd) * 16);
+                rec[0] = make_uint4(d0, d1, 0u, 0u);  // even A rows
+                rec[1] = make_uint4(0u, 0u, d0, d1);  // odd A rows
             }
         }
+        if (threadIdx.x == 0)
+            *reinterpret_cast<uint4 *>(zero_rec) = make_uint4(0u, 0u, 0u, 0u);
     }
     __syncthreads();
 
@@ -311,13 +319,39 @@ __global__ void __launch_bounds__(kGemvThreads, MG == 1 ? 2 : 1) gemv_kernel(con
         if (*flag != 1)
             return;
         __threadfence();
-        for (int e = tid; e < m * 128; e += kGemvThreads) {
+        // sum the partials in split order; eight independent loads in flight
+        // per thread, and for m = 1 two threads per element (even / odd
+        // splits) combined afterwards, so the L2 latency is paid a few times
+        // rather than once per split
+        const int E = m * 128;
+        const int per_elem = E < kGemvThreads ? 2 : 1;
+        float *part2 = red + E;  // second-half sums when per_elem == 2
+        for (int u = tid; u < E * per_elem; u += kGemvThreads) {
+            const int e = u % E, h = u / E;
             const int b = e >> 7, c = e & 127;
-            float sum = 0.f;
-            for (int sp = 0; sp < p.splits; ++sp)
-                sum += __ldcg(&p.partials[((int64_t)sp * m + b) * n + nb * 128 + c]);
-            red[e] = sum;
+            const float *src = p.partials + (int64_t)b * n + nb * 128 + c;
+            const int64_t sstride = (int64_t)m * n;
+            float acc8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            int sp = h;
+            for (; sp + 7 * per_elem < p.splits; sp += 8 * per_elem) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    acc8[i] += __ldcg(src + (int64_t)(sp + i * per_elem) * sstride);
+            }
+            float tail = 0.f;
+            for (; sp < p.splits; sp += per_elem)
+                tail += __ldcg(src + (int64_t)sp * sstride);
+            const float sum =
+                (((acc8[0] + acc8[1]) + (acc8[2] + acc8[3])) + ((acc8[4] + acc8[5]) + (acc8[6] + acc8[7]))) + tail;
+            if (h == 0)
+                red[e] = sum;
+            else
+                part2[e] = sum;
         }
+        __syncthreads();
+        if (per_elem == 2)
+            for (int e = tid; e < E; e += kGemvThreads)
+                red[e] += part2[e];
         if (tid == 0)
             p.counters[nb] = 0u;
         __syncthreads();
