@@ -116,6 +116,36 @@ exl3_status exl3_gemv(const void *x, const uint16_t *trellis, const void *suh, c
                       size_t workspace_bytes, void *stream);
 
 /*
+ * exl3_gemv_noalloc -- exl3_gemv for callers that cannot allocate device
+ * memory.  (The pages have no counterpart: this is a library convenience.)
+ *
+ * Some callers cannot call cudaMalloc or an allocator of their own: code that
+ * runs under a host framework which owns all device memory, a plugin with a
+ * fixed memory budget, or a latency-critical path where an allocation (and the
+ * device synchronisation it may imply) is not allowed.  This entry point needs
+ * no workspace argument: its scratch (split-k partial sums and arrival
+ * counters) is a fixed array of exl3_gemv_noalloc_max_scratch() bytes (4 MiB)
+ * compiled into the library, which every GPU that loads the library holds
+ * until the process exits.  The caller still passes x, the weights and y.
+ *   - Shapes whose scratch exceeds that maximum are rejected with
+ *     EXL3_ERR_WORKSPACE before anything is launched (exl3_gemv_workspace_size
+ *     tells how much a shape needs).
+ *   - The first call on a device looks the array's device address up
+ *     (cudaGetSymbolAddress) and caches it; make that first call before any
+ *     stream capture on that device.
+ *   - Every call on a device shares the one array and it keeps the last call's
+ *     contents: each call first clears the arrival counters on its stream, and
+ *     calls that can overlap on the GPU (different streams, or concurrent
+ *     host threads) race on the array and must not be issued.
+ *   - No cudaMalloc, cudaFree or other allocating routine is called.
+ * Arguments and results otherwise as exl3_gemv.
+ */
+size_t exl3_gemv_noalloc_max_scratch(void);
+exl3_status exl3_gemv_noalloc(const void *x, const uint16_t *trellis, const void *suh,
+                              const void *svh, void *y, int64_t m, int64_t k, int64_t n, int K,
+                              void *stream);
+
+/*
  * exl3_gemm -- the linear layer on the tensor cores (tcgen05 / TMEM), any
  * m >= 1, tuned for m >= 64 ([GEMM] section GEMM内核: Hadamard rotation of the
  * input, then the dequantising matmul; the kernel map picks tiles by shape).

@@ -522,3 +522,78 @@ extern "C" exl3_status exl3_gemv(const void *x, const uint16_t *trellis, const v
     return run_gemv(x, trellis, suh, svh, y, m, k, n, K, workspace, workspace_bytes,
                     (cudaStream_t)stream);
 }
+
+// ------------------------------------------------ no-allocation variant ---
+//
+// exl3_gemv_noalloc runs the GEMV above with its scratch (split-k partials
+// and arrival counters) in a fixed array compiled into the library, for
+// callers that must not allocate device memory themselves.  The array is a
+// file-scope __device__ symbol: every GPU that loads the library holds its
+// kNoAllocScratchBytes until the process exits.  In host code the symbol's
+// name is only a host-side stand-in, so the device address is looked up once
+// per device with cudaGetSymbolAddress (with that device current) and cached.
+
+#include <mutex>
+
+namespace exl3 {
+
+constexpr size_t kNoAllocScratchBytes = 4u << 20;  // 4 MiB per device
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+static void *g_noalloc_ptr[kMaxDevices];
+static std::mutex g_noalloc_mutex;
+
+// Device address of this device's scratch array (set up on first use).
+static exl3_status noalloc_scratch(void **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return EXL3_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices)
+        return EXL3_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)
+            return EXL3_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return EXL3_OK;
+}
+
+}  // namespace exl3
+
+extern "C" size_t exl3_gemv_noalloc_max_scratch(void)
+{
+    return exl3::kNoAllocScratchBytes;
+}
+
+extern "C" exl3_status exl3_gemv_noalloc(const void *x, const uint16_t *trellis, const void *suh,
+                                         const void *svh, void *y, int64_t m, int64_t k, int64_t n,
+                                         int K, void *stream)
+{
+    using namespace exl3;
+    const exl3_status st = check_linear_args(x, trellis, suh, svh, y, m, k, n, K);
+    if (st != EXL3_OK)
+        return st;
+    if (m > 16)
+        return EXL3_ERR_UNSUPPORTED;
+    const size_t need = gemv_workspace_bytes(m, k, n, num_sms());
+    if (need > kNoAllocScratchBytes)
+        return EXL3_ERR_WORKSPACE;  // this shape needs more scratch than the built-in array
+    void *scratch = nullptr;
+    const exl3_status sst = noalloc_scratch(&scratch);
+    if (sst != EXL3_OK)
+        return sst;
+    // the array keeps whatever the last call left: the arrival counters must
+    // start at zero (the kernel re-arms them, but a call that never finished
+    // could have left them set), so clear them on the caller's stream
+    const size_t counter_bytes = 256 + (size_t)((n / 128) * 4 + 255) / 256 * 256;
+    if (cudaMemsetAsync(scratch, 0, counter_bytes, (cudaStream_t)stream) != cudaSuccess)
+        return EXL3_ERR_CUDA;
+    return run_gemv(x, trellis, suh, svh, y, m, k, n, K, scratch, kNoAllocScratchBytes,
+                    (cudaStream_t)stream);
+}

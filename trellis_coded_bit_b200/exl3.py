@@ -22,7 +22,8 @@ EXL3_ERR_TIMEOUT = 5
 
 # Every symbol the public headers declare.
 EXPORTED = ["exl3_status_string", "exl3_version", "exl3_hadamard", "exl3_decode_tiles",
-            "exl3_gemv_workspace_size", "exl3_gemv", "exl3_gemm_workspace_size", "exl3_gemm",
+            "exl3_gemv_workspace_size", "exl3_gemv", "exl3_gemv_noalloc_max_scratch",
+            "exl3_gemv_noalloc", "exl3_gemm_workspace_size", "exl3_gemm",
             "exl3_workspace_status", "exl3_set_launch_flags", "exl3_launch_flags",
             "exl3_debug_set_wait_limit_ns", "exl3_debug_wait_limit_ns"]
 
@@ -68,6 +69,10 @@ def load(build_if_needed=True):
         for name in ("exl3_gemv", "exl3_gemm"):
             getattr(lib, name).argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, ci, vp, sz, vp]
             getattr(lib, name).restype = ci
+        lib.exl3_gemv_noalloc_max_scratch.argtypes = []
+        lib.exl3_gemv_noalloc_max_scratch.restype = sz
+        lib.exl3_gemv_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, ci, vp]
+        lib.exl3_gemv_noalloc.restype = ci
         lib.exl3_workspace_status.argtypes = [vp, sz, ci, vp]
         lib.exl3_workspace_status.restype = ci
         lib.exl3_set_launch_flags.argtypes = [ctypes.c_uint]
@@ -168,6 +173,22 @@ def _linear(fn, name, x, trellis, suh, svh, K, y, workspace, stream):
 def exl3_gemv(x, trellis, suh, svh, K, y=None, workspace=None, stream=None):
     """y = svh .* H(H(x .* suh) W_hat) for 1 <= m <= 16 (memory-bound path)."""
     return _linear(load().exl3_gemv, "exl3_gemv", x, trellis, suh, svh, K, y, workspace, stream)
+
+
+def exl3_gemv_noalloc_max_scratch():
+    return int(load().exl3_gemv_noalloc_max_scratch())
+
+
+def exl3_gemv_noalloc(x, trellis, suh, svh, K, y, stream=None):
+    """exl3_gemv without a workspace: the library's own fixed scratch array is
+    used, for callers that cannot allocate device memory (y must be given)."""
+    m, k = x.shape
+    n = svh.numel()
+    _check(load().exl3_gemv_noalloc(_dev(x, torch.float16, "x"), _dev(trellis, torch.uint16, "trellis"),
+                                    _dev(suh, torch.float16, "suh"), _dev(svh, torch.float16, "svh"),
+                                    _dev(y, torch.float16, "y"), m, k, n, int(K), _stream(stream)),
+           "exl3_gemv_noalloc")
+    return y
 
 
 def exl3_gemm(x, trellis, suh, svh, K, y=None, workspace=None, stream=None):
