@@ -158,50 +158,97 @@ __device__ __forceinline__ int row_of(int q, int t)
     return 2 * (4 * (q & 1) + t) + (q >> 1);
 }
 
+// Per-warp shared-memory ring: each stage holds one unit -- the 8 tiles of a
+// tile row (each padded to 32K + 16 bytes, which spreads the lanes' row reads
+// over the banks) and that tile row's 16 x slots activation records.
 template <int K>
-struct RowBuf {
-    static constexpr int N =
-        RowSpan<K, 0>::N32 > RowSpan<K, 1>::N32 ? RowSpan<K, 0>::N32 : RowSpan<K, 1>::N32;
-    uint32_t w[4][N];
+struct Stage {
+    static constexpr int kTileStride = 32 * K + 16;
+    static constexpr int kTileBytes = 8 * kTileStride;
 };
 
-template <int K>
-__device__ __forceinline__ void load_tile_row(const uint32_t *tile, int t, RowBuf<K> &b)
+__host__ __device__ inline int gemv_stage_bytes(int K, int m)
 {
-    load_row<K, 0>(tile, row_of(0, t), b.w[0]);
-    load_row<K, 0>(tile, row_of(1, t), b.w[1]);
-    load_row<K, 1>(tile, row_of(2, t), b.w[2]);
-    load_row<K, 1>(tile, row_of(3, t), b.w[3]);
+    return 8 * (32 * K + 16) + 16 * rec_slots(m) * 16 + 16;  // tiles, records, zero record
 }
 
-// Activation-record address of one lane for one batch group (the zero
-// record, stride 0, when the lane's quad holds no batch).
-struct RecPtr {
-    const unsigned char *base;
-    int stride;
+constexpr int kGemvDepth = 3;  // units in flight per warp (one consumed, two loading)
+
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_addr(smem_dst)), "l"(gsrc)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit()
+{
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait()
+{
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+// Per-lane, per-row-group constants: byte offsets (within a stage) of the
+// lane's prefix word, of its row's first 32-bit word, and of its activation
+// record(s) -- the lane's rows never change, so these are computed once.
+struct LaneRows {
+    int pre[4], row[4];
+    int rec[4][2];  // [q][mg] (offset of the record, or of the stage's zero record)
 };
 
+// Loads a tile row from shared memory at precomputed offsets, as wide as the
+// row's alignment allows (K = 4: 8 bytes, K = 8: 16 bytes).
+template <int K, int PAR, int N>
+__device__ __forceinline__ void load_row_at(const unsigned char *stage, int pre, int row, uint32_t (&raw)[N])
+{
+    constexpr int P = RowSpan<K, PAR>::P;
+    constexpr int N32 = RowSpan<K, PAR>::N32;
+    raw[0] = *reinterpret_cast<const uint32_t *>(stage + pre);
+    if constexpr (K == 4 && P == 1) {
+        const uint2 v = *reinterpret_cast<const uint2 *>(stage + row);
+        raw[1] = v.x;
+        raw[2] = v.y;
+    } else if constexpr (K == 8 && P == 1) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(stage + row);
+        raw[1] = v.x;
+        raw[2] = v.y;
+        raw[3] = v.z;
+        raw[4] = v.w;
+    } else {
+#pragma unroll
+        for (int i = 1; i < N32; ++i)
+            raw[i] = *reinterpret_cast<const uint32_t *>(stage + row + 4 * (i - 1));
+    }
+}
+
 template <int K, int MG>
-__device__ __forceinline__ void mac_tile_row(const RowBuf<K> &buf, int kk0, const RecPtr (&rp)[MG], int t,
-                                             const Codebook &cb, float (&acc)[MG][8][4])
+__device__ __forceinline__ void mac_stage(const unsigned char *stage, const LaneRows &lr, const Codebook &cb,
+                                          float (&acc)[MG][8][4])
 {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-        const int kk = kk0 + row_of(q, t);
         uint32_t A[MG][4];
 #pragma unroll
         for (int mg = 0; mg < MG; ++mg) {
-            const uint4 r = __ldg(reinterpret_cast<const uint4 *>(rp[mg].base + (int64_t)kk * rp[mg].stride));
+            const uint4 r = *reinterpret_cast<const uint4 *>(stage + lr.rec[q][mg]);
             A[mg][0] = r.x;
             A[mg][1] = r.y;
             A[mg][2] = r.z;
             A[mg][3] = r.w;
         }
         uint32_t s[16];
-        if (q < 2)
-            row_states<K, RowSpan<K, 0>::P>(buf.w[q], s);
-        else
-            row_states<K, RowSpan<K, 1>::P>(buf.w[q], s);
+        if (q < 2) {
+            uint32_t raw[RowSpan<K, 0>::N32];
+            load_row_at<K, 0>(stage, lr.pre[q], lr.row[q], raw);
+            row_states<K, RowSpan<K, 0>::P>(raw, s);
+        } else {
+            uint32_t raw[RowSpan<K, 1>::N32];
+            load_row_at<K, 1>(stage, lr.pre[q], lr.row[q], raw);
+            row_states<K, RowSpan<K, 1>::P>(raw, s);
+        }
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const uint32_t b0 = codebook_word(s[2 * j], cb);
@@ -211,15 +258,6 @@ __device__ __forceinline__ void mac_tile_row(const RowBuf<K> &buf, int kk0, cons
                 mma_16816(acc[mg][j], A[mg], b0, b1);
         }
     }
-}
-
-// Unit u -> its tiles for lane g: column block cb = u / tr_count, tile row
-// tr = u % tr_count.
-__device__ __forceinline__ const uint32_t *unit_tiles(const GemvParams &p, int64_t u, int g, int K)
-{
-    const int64_t cb = u / p.tr_count, tr = u - cb * p.tr_count;
-    return reinterpret_cast<const uint32_t *>(p.trellis) +
-           ((tr * (p.n >> 4) + cb * 8 + g) * 8 * (int64_t)K);
 }
 
 // CTA owning unit u: the largest c with floor(c U / G) <= u.
@@ -253,75 +291,96 @@ __device__ __forceinline__ void finish_block(const GemvParams &p, const float *r
 template <int K, int MG>
 __global__ void __launch_bounds__(kGemvThreads, MG == 1 ? 2 : 1) gemv_kernel(const GemvParams p)
 {
-    extern __shared__ __align__(16) unsigned char smem[];
+    extern __shared__ __align__(128) unsigned char smem[];
     volatile int *flag = reinterpret_cast<volatile int *>(smem);
-    float *red = reinterpret_cast<float *>(smem + 16);  // [warps][m][128], row 0 reused for sums
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = lane >> 2, t = lane & 3;
     const int m = p.m;
+    const int slots = rec_slots(m);
+    const int stage_bytes = (gemv_stage_bytes(K, m) + 127) & ~127;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    unsigned char *ring = smem + 128 + warp * kGemvDepth * stage_bytes;
+    float *red = reinterpret_cast<float *>(smem + 128 + kGemvWarps * kGemvDepth * stage_bytes);
+
+    const int g = lane >> 2, t = lane & 3;
+    const int TR = p.tr_count;
     const int64_t U = p.units;
     const int G = p.ctas;
     const int64_t u0 = (int64_t)blockIdx.x * U / G, u1 = (int64_t)(blockIdx.x + 1) * U / G;
-    const int TR = p.tr_count;
-
-    // this warp's unit sequence: the CTA's segments in order, inside each the
-    // tile rows warp, warp+8, ...  Start the first two loads right away.
-    auto next_unit = [&](int64_t u) -> int64_t {
-        // the unit after u in this warp's sequence, or u1 when done
-        const int64_t cb = u / TR;
-        const int64_t seg_end = (cb + 1) * TR < u1 ? (cb + 1) * TR : u1;
-        if (u + kGemvWarps < seg_end)
-            return u + kGemvWarps;
-        // next segment: its first unit plus this warp's offset
-        int64_t nb = seg_end;
-        while (nb < u1) {
-            const int64_t e = ((nb / TR) + 1) * TR < u1 ? ((nb / TR) + 1) * TR : u1;
-            if (nb + warp < e)
-                return nb + warp;
-            nb = e;
+    // the range as column blocks [cb0, cb1], first block from tile row tb0,
+    // last block up to (excluding) tile row te1
+    const int cb0 = (int)(u0 / TR), tb0 = (int)(u0 - (int64_t)cb0 * TR);
+    const int cb1 = (int)((u1 - 1) / TR), te1 = (int)(u1 - (int64_t)cb1 * TR);
+    auto seg_tb = [&](int c) { return c == cb0 ? tb0 : 0; };
+    auto seg_te = [&](int c) { return c == cb1 ? te1 : TR; };
+    // first unit of this warp at or after column block c (cb > cb1: none)
+    auto first_from = [&](int c, int &tr_out) {
+        for (; c <= cb1; ++c) {
+            const int tr = seg_tb(c) + warp;
+            if (tr < seg_te(c)) {
+                tr_out = tr;
+                return c;
+            }
         }
-        return u1;
+        tr_out = 0;
+        return cb1 + 1;
     };
-    auto first_unit = [&]() -> int64_t {
-        int64_t nb = u0;
-        while (nb < u1) {
-            const int64_t e = ((nb / TR) + 1) * TR < u1 ? ((nb / TR) + 1) * TR : u1;
-            if (nb + warp < e)
-                return nb + warp;
-            nb = e;
-        }
-        return u1;
+    auto advance = [&](int &c, int &tr) {
+        tr += kGemvWarps;
+        if (tr >= seg_te(c))
+            c = first_from(c + 1, tr);
     };
 
-    RowBuf<K> buf0, buf1;
-    int64_t ua = first_unit();
-    int64_t ub = ua < u1 ? next_unit(ua) : u1;
-    if (ua < u1)
-        load_tile_row<K>(unit_tiles(p, ua, g, K), t, buf0);
-    if (ub < u1)
-        load_tile_row<K>(unit_tiles(p, ub, g, K), t, buf1);
-    const Codebook cb = p.cb;
+    const int64_t tile_row_bytes = (int64_t)(p.n >> 4) * 32 * K;  // one tile row of the matrix
+    const int rec_row_bytes = 16 * slots * 16;                   // records of one tile row
+    auto issue = [&](int c, int tr, unsigned char *stage) {
+        if (c <= cb1) {
+            const unsigned char *src =
+                reinterpret_cast<const unsigned char *>(p.trellis) + tr * tile_row_bytes + (int64_t)c * 8 * 32 * K;
+            for (int i = lane; i < 16 * K; i += 32)
+                cp_async16(stage + (i / (2 * K)) * Stage<K>::kTileStride + (i % (2 * K)) * 16, src + i * 16);
+            const unsigned char *rsrc = p.recs + (int64_t)tr * rec_row_bytes;
+            for (int i = lane; i < 16 * slots; i += 32)
+                cp_async16(stage + Stage<K>::kTileBytes + i * 16, rsrc + i * 16);
+        }
+        cp_async_commit();
+    };
 
-    // records and the workspace are written by the rotation kernel / other
-    // launches: wait for the preceding kernel (no-op without PDL)
-    grid_dep_wait();
-
-    const int slots = rec_slots(m);
-    RecPtr rp[MG];
+    // per-lane offsets within a stage
+    LaneRows lr;
 #pragma unroll
-    for (int mg = 0; mg < MG; ++mg) {
-        const int ba = g >> 1;
-        const int qbase = mg * rec_quads(m, 0);
-        if (ba < rec_quads(m, mg)) {
-            rp[mg].base = p.recs + (2 * (qbase + ba) + (g & 1)) * 16;
-            rp[mg].stride = slots * 16;
-        } else {
-            rp[mg].base = p.zero_rec;
-            rp[mg].stride = 0;
+    for (int q = 0; q < 4; ++q) {
+        const int rho = row_of(q, t);
+        const int first = (rho * K - 1) >> 1;  // -1 for row 0: the tile's last word (wrap)
+        lr.pre[q] = g * Stage<K>::kTileStride + 4 * (first < 0 ? 8 * K - 1 : first);
+        lr.row[q] = g * Stage<K>::kTileStride + 4 * (first + 1);
+#pragma unroll
+        for (int mg = 0; mg < 2; ++mg) {
+            const int ba = g >> 1;
+            const bool have = mg < MG && ba < rec_quads(m, mg);
+            const int slot = 2 * (mg * rec_quads(m, 0) + ba) + (g & 1);
+            lr.rec[q][mg] = have ? Stage<K>::kTileBytes + (rho * slots + slot) * 16
+                                 : Stage<K>::kTileBytes + rec_row_bytes;  // zero record
         }
     }
 
+    // the zero record of every stage of this warp's ring
+    if (lane < kGemvDepth)
+        *reinterpret_cast<uint4 *>(ring + lane * stage_bytes + Stage<K>::kTileBytes + rec_row_bytes) =
+            make_uint4(0u, 0u, 0u, 0u);
+
+    // records come from the rotation kernel: wait for it (no-op without PDL)
+    grid_dep_wait();
+    int ci, ti;  // issue iterator, kGemvDepth units ahead of consumption
+    ci = first_from(cb0, ti);
+    int cc = ci, tc = ti;  // consume iterator
+#pragma unroll
+    for (int d = 0; d < kGemvDepth; ++d) {
+        issue(ci, ti, ring + d * stage_bytes);
+        if (ci <= cb1)
+            advance(ci, ti);
+    }
+    __syncwarp();
+
+    const Codebook cb = p.cb;
     float acc[MG][8][4];
 #pragma unroll
     for (int a = 0; a < MG; ++a)
@@ -331,31 +390,24 @@ __global__ void __launch_bounds__(kGemvThreads, MG == 1 ? 2 : 1) gemv_kernel(con
             for (int e = 0; e < 4; ++e)
                 acc[a][j][e] = 0.f;
 
-    // segments of this CTA, in order; buffer `phase` holds unit ua, the other
-    // one unit ub (both loaded or in flight)
-    int phase = 0;
-    int64_t seg_begin = u0;
-    while (seg_begin < u1) {
-        const int cbk = (int)(seg_begin / TR);
-        const int64_t seg_end = ((int64_t)cbk + 1) * TR < u1 ? ((int64_t)cbk + 1) * TR : u1;
-        while (ua < seg_end) {
-            const int64_t uc = ub < u1 ? next_unit(ub) : u1;
-            const int kk0 = (int)(ua - (int64_t)cbk * TR) * 16;
-            if (phase == 0) {
-                mac_tile_row<K, MG>(buf0, kk0, rp, t, cb, acc);
-                if (uc < u1)
-                    load_tile_row<K>(unit_tiles(p, uc, g, K), t, buf0);
-            } else {
-                mac_tile_row<K, MG>(buf1, kk0, rp, t, cb, acc);
-                if (uc < u1)
-                    load_tile_row<K>(unit_tiles(p, uc, g, K), t, buf1);
-            }
-            phase ^= 1;
-            ua = ub;
-            ub = uc;
+    int st = 0;
+    for (int cbk = cb0; cbk <= cb1; ++cbk) {
+        while (cc == cbk) {
+            cp_async_wait<kGemvDepth - 1>();
+            __syncwarp();
+            unsigned char *stage = ring + st * stage_bytes;
+            mac_stage<K, MG>(stage, lr, cb, acc);
+            __syncwarp();  // every lane is done with the stage before it is refilled
+            issue(ci, ti, stage);
+            if (ci <= cb1)
+                advance(ci, ti);
+            st = st + 1 == kGemvDepth ? 0 : st + 1;
+            advance(cc, tc);
         }
+        const int64_t seg_begin = (int64_t)cbk * TR + seg_tb(cbk);
+        const int64_t seg_end = (int64_t)cbk * TR + seg_te(cbk);
 
-        // ------------------------------------------- segment end: reduce ---
+    // ------------------------------------------- segment end: reduce ---
         // accumulator (mg, j, e): A row i = g (+8 for e >= 2) -> batch 8mg + i/2,
         // column parity i&1; n-slot 2t (+1 for odd e) -> tile of the block;
         // column = 16 * slot + 2j + parity.
@@ -415,8 +467,8 @@ __global__ void __launch_bounds__(kGemvThreads, MG == 1 ? 2 : 1) gemv_kernel(con
             }
         }
         __syncthreads();  // red is reused by the next segment
-        seg_begin = seg_end;
     }
+    cp_async_wait<0>();  // nothing may still be landing in shared memory at exit
 }
 
 // ------------------------------------------------------------- dispatch ---
@@ -448,14 +500,22 @@ static int64_t owner_cta_host(int64_t u, int64_t U, int64_t G)
     return ((u + 1) * G - 1) / U;
 }
 
-// Grid: all resident CTAs (2 per SM for m <= 8, 1 above) but at least two
-// units per warp; max_seg = the most CTAs any column block is split over.
-static GemvPlan gemv_plan(int64_t m, int64_t k, int64_t n, int sms)
+// Grid: every CTA resident at once -- resident CTAs per SM from the register
+// budget (2 for m <= 8, 1 above) and the shared memory (228 KB per SM, 1 KB
+// reserved per CTA) -- but at least two units per warp; max_seg = the most
+// CTAs any column block is split over.
+static GemvPlan gemv_plan(int64_t m, int64_t k, int64_t n, int K, int sms)
 {
     GemvPlan pl;
     const int64_t TR = k / 16, ncb = n / 128;
     pl.units = TR * ncb;
-    int64_t G = (m <= 8 ? 2 : 1) * (int64_t)sms;
+    pl.smem = 128 + kGemvWarps * kGemvDepth * ((gemv_stage_bytes(K, (int)m) + 127) & ~127) +
+              kGemvWarps * (int)m * 128 * 4;
+    int64_t occ = m <= 8 ? 2 : 1;
+    const int64_t occ_smem = (228 * 1024) / (pl.smem + 1024);
+    if (occ_smem < occ)
+        occ = occ_smem > 0 ? occ_smem : 1;
+    int64_t G = occ * (int64_t)sms;
     const int64_t gmax = pl.units / (2 * kGemvWarps);
     if (G > gmax)
         G = gmax > 0 ? gmax : 1;
@@ -467,14 +527,18 @@ static GemvPlan gemv_plan(int64_t m, int64_t k, int64_t n, int sms)
             max_seg = s;
     }
     pl.max_seg = (int)max_seg;
-    pl.smem = 16 + kGemvWarps * (int)m * 128 * 4;
     return pl;
 }
 
 size_t gemv_workspace_bytes(int64_t m, int64_t k, int64_t n, int sms)
 {
-    const GemvPlan pl = gemv_plan(m, k, n, sms);
-    return gemv_layout(m, k, n, pl.max_seg).total;
+    size_t most = 0;
+    for (int K = 1; K <= 8; ++K) {
+        const GemvPlan pl = gemv_plan(m, k, n, K, sms);
+        const size_t b = gemv_layout(m, k, n, pl.max_seg).total;
+        most = b > most ? b : most;
+    }
+    return most;
 }
 
 template <int K, int MG>
@@ -509,7 +573,7 @@ exl3_status run_gemv(const void *x, const uint16_t *trellis, const void *suh, co
                      size_t workspace_bytes, cudaStream_t stream)
 {
     const int sms = num_sms();
-    const GemvPlan pl = gemv_plan(m, k, n, sms);
+    const GemvPlan pl = gemv_plan(m, k, n, K, sms);
     const GemvLayout L = gemv_layout(m, k, n, pl.max_seg);
     if (!workspace || !aligned16(workspace) || workspace_bytes < L.total)
         return EXL3_ERR_WORKSPACE;
