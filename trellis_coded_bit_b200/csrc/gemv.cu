@@ -335,11 +335,20 @@ __global__ void __launch_bounds__(kGemvThreads, MG == 1 ? 2 : 1) gemv_kernel(con
         if (c <= cb1) {
             const unsigned char *src =
                 reinterpret_cast<const unsigned char *>(p.trellis) + tr * tile_row_bytes + (int64_t)c * 8 * 32 * K;
-            for (int i = lane; i < 16 * K; i += 32)
-                cp_async16(stage + (i / (2 * K)) * Stage<K>::kTileStride + (i % (2 * K)) * 16, src + i * 16);
+            // 16K chunks of 16 bytes: tile i / 2K, chunk i % 2K
+#pragma unroll
+            for (int r = 0; r < (16 * K + 31) / 32; ++r) {
+                const int i = lane + 32 * r;
+                if ((16 * K) % 32 == 0 || i < 16 * K)
+                    cp_async16(stage + (i / (2 * K)) * Stage<K>::kTileStride + (i % (2 * K)) * 16, src + i * 16);
+            }
             const unsigned char *rsrc = p.recs + (int64_t)tr * rec_row_bytes;
-            for (int i = lane; i < 16 * slots; i += 32)
-                cp_async16(stage + Stage<K>::kTileBytes + i * 16, rsrc + i * 16);
+#pragma unroll
+            for (int r = 0; r < 4 * MG; ++r) {  // up to 16 x 8 slots per batch group
+                const int i = lane + 32 * r;
+                if (i < 16 * slots)
+                    cp_async16(stage + Stage<K>::kTileBytes + i * 16, rsrc + i * 16);
+            }
         }
         cp_async_commit();
     };
@@ -454,11 +463,18 @@ __global__ void __launch_bounds__(kGemvThreads, MG == 1 ? 2 : 1) gemv_kernel(con
             __syncthreads();
             if (*flag == 1) {
                 __threadfence();
+                // segment order, eight independent loads in flight per thread
                 for (int e = tid; e < m * 128; e += kGemvThreads) {
-                    float sum = 0.f;
-                    for (int s2 = 0; s2 < nseg; ++s2)
-                        sum += __ldcg(part + (int64_t)s2 * m * 128 + e);
-                    red[e] = sum;
+                    float a8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    int s2 = 0;
+                    for (; s2 + 8 <= nseg; s2 += 8)
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            a8[i] += __ldcg(part + (int64_t)(s2 + i) * m * 128 + e);
+                    float tail = 0.f;
+                    for (; s2 < nseg; ++s2)
+                        tail += __ldcg(part + (int64_t)s2 * m * 128 + e);
+                    red[e] = (((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]))) + tail;
                 }
                 if (tid == 0)
                     p.counters[cbk] = 0u;
