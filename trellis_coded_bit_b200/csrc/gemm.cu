@@ -41,7 +41,7 @@ constexpr int kBM = 128;             // rows per MMA tile (TMEM lanes)
 constexpr int kMT = 4;               // M tiles per CTA sharing one decoded B
 constexpr int kBN = 128;             // output channels per CTA (MMA N) = one Hadamard block
 constexpr int kBK = 32;              // input channels per stage
-constexpr int kDecWarps = 4;         // decoder warps, also the epilogue warps
+constexpr int kDecWarps = 8;         // decoder warps; the first four are also the epilogue
 constexpr int kGemmThreads = 32 * (2 + kDecWarps);
 constexpr int kATileBytes = kBM * kBK * 2;   // 8 KB: K-major, 64-byte rows, 64-byte swizzle
 constexpr int kBTileBytes = kBK * kBN * 2;   // 8 KB: MN-major, 128-byte swizzle
@@ -396,16 +396,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmParams 
             unsigned char *st = stages + s * kStage;
             unsigned char *bt = st + kMT * kATileBytes;
             const unsigned char *tr = bt + kBTileBytes;
-            // 4 tiles per warp; lane l decodes rows 2(l%8) and 2(l%8)+1 of tile
-            // l/8 (one parity per pass: compile-time bit windows)
-            static_assert((kBK / 16) * (kBN / 16) == 4 * kDecWarps, "tiles per stage");
+            // decoder warp dw takes tiles 4(dw/2) .. 4(dw/2)+3 and the rows of
+            // parity dw%2 (compile-time bit windows): lane l decodes row
+            // 2(l%8) + dw%2 of tile 4(dw/2) + l/8
+            static_assert((kBK / 16) * (kBN / 16) == 2 * kDecWarps, "tiles per stage");
             {
-                const int T = dw * 4 + (lane >> 3);
+                const int T = (dw >> 1) * 4 + (lane >> 3);
                 const int trow = T / (kBN / 16), tcol = T - (T / (kBN / 16)) * (kBN / 16);
                 const uint32_t *tw = reinterpret_cast<const uint32_t *>(tr + T * 32 * K);
                 const int r0 = 2 * (lane & 7);
-                decode_row_to_b<K, 0>(tw, r0, p.cb, bt, trow, tcol);
-                decode_row_to_b<K, 1>(tw, r0 + 1, p.cb, bt, trow, tcol);
+                if (dw & 1)
+                    decode_row_to_b<K, 1>(tw, r0 + 1, p.cb, bt, trow, tcol);
+                else
+                    decode_row_to_b<K, 0>(tw, r0, p.cb, bt, trow, tcol);
             }
             fence_proxy_async_smem();
             __syncwarp();
