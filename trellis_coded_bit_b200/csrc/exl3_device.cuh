@@ -182,10 +182,13 @@ __device__ __forceinline__ void row_weights_f16(const uint32_t (&raw)[N], const 
     for (int j = 0; j < 8; ++j) {
         const uint32_t v0 = codebook_word(s[2 * j], cb);
         const uint32_t v1 = codebook_word(s[2 * j + 1], cb);
-        const uint32_t lo = __byte_perm(v0, v1, 0x5410u);  // low halves of both words
-        const uint32_t hi = __byte_perm(v0, v1, 0x7632u);  // high halves of both words
-        __half2 w = __hadd2(*reinterpret_cast<const __half2 *>(&lo), *reinterpret_cast<const __half2 *>(&hi));
-        out[j] = *reinterpret_cast<uint32_t *>(&w);
+        const __half2 h0 = *reinterpret_cast<const __half2 *>(&v0);
+        const __half2 h1 = *reinterpret_cast<const __half2 *>(&v1);
+        // lo + hi of each word in both lanes (one add with half selects), then
+        // one byte permute packs the two weights
+        __half2 w0 = __hadd2(__low2half2(h0), __high2half2(h0));
+        __half2 w1 = __hadd2(__low2half2(h1), __high2half2(h1));
+        out[j] = __byte_perm(*reinterpret_cast<uint32_t *>(&w0), *reinterpret_cast<uint32_t *>(&w1), 0x5410u);
     }
 }
 

@@ -38,13 +38,13 @@
 namespace exl3 {
 
 constexpr int kBM = 128;             // rows per MMA tile (TMEM lanes)
-constexpr int kMT = 4;               // M tiles per CTA sharing one decoded B
-constexpr int kBN = 128;             // output channels per CTA (MMA N) = one Hadamard block
-constexpr int kBK = 32;              // input channels per stage
-constexpr int kDecWarps = 8;         // decoder warps; the first four are also the epilogue
+constexpr int kMT = 2;               // M tiles per CTA sharing one decoded B
+constexpr int kBN = 256;             // output channels per CTA (MMA N)
+constexpr int kBK = 64;              // input channels per stage
+constexpr int kDecWarps = 16;
 constexpr int kGemmThreads = 32 * (2 + kDecWarps);
-constexpr int kATileBytes = kBM * kBK * 2;   // 8 KB: K-major, 64-byte rows, 64-byte swizzle
-constexpr int kBTileBytes = kBK * kBN * 2;   // 8 KB: MN-major, 128-byte swizzle
+constexpr int kATileBytes = kBM * kBK * 2;   // 16 KB
+constexpr int kBTileBytes = kBK * kBN * 2;   // 32 KB
 constexpr int kTmemCols = kMT * kBN;         // 512
 
 __host__ __device__ constexpr int gemm_trellis_stage_bytes(int K)
@@ -59,7 +59,7 @@ __host__ __device__ constexpr int gemm_stage_bytes(int K)
 
 __host__ __device__ constexpr int gemm_stages(int K)
 {
-    return (220 * 1024) / gemm_stage_bytes(K) >= 6 ? 6 : (220 * 1024) / gemm_stage_bytes(K);
+    return (220 * 1024) / gemm_stage_bytes(K) >= 3 ? 3 : 2;
 }
 
 __host__ __device__ constexpr int gemm_smem_bytes(int K)
@@ -160,13 +160,11 @@ __device__ __forceinline__ void tmem_wait_st()
     asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
 }
 
-// Shared-memory matrix descriptor, sm_100 format; layout 2 = 128-byte
-// swizzle, 4 = 64-byte swizzle.
-constexpr uint32_t kSw128 = 2, kSw64 = 4;
-__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout)
+// Shared-memory matrix descriptor: 128-byte swizzle, sm_100 format.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo)
 {
     return (uint64_t)((saddr >> 4) & 0x3fffu) | ((uint64_t)((lbo >> 4) & 0x3fffu) << 16) |
-           ((uint64_t)((sbo >> 4) & 0x3fffu) << 32) | (1ull << 46) | ((uint64_t)layout << 61);
+           ((uint64_t)((sbo >> 4) & 0x3fffu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
 // Instruction descriptor, kind::f16: D f32, A f16 K-major, B f16 MN-major.
@@ -193,9 +191,7 @@ __device__ __forceinline__ void fwht32(float (&v)[32])
 // -------------------------------------------------------- rotation pass ---
 
 // x'[r, :] = H(x[r, :] .* suh)/sqrt(128) written in the tiled, swizzled A
-// layout: tile (r/128, c/32) of 8 KB, 64-byte row r%128, 16-byte chunk
-// ((c%32)/8) ^ ((r%128 / 2) % 4) -- the tensor core's canonical K-major
-// layout with 64-byte swizzle (8-row atoms of 512 bytes).
+// layout: tile (r/128, c/64), 128-byte row r%128, 16-byte chunk ((c%64)/8) ^ (r%8).
 __global__ void __launch_bounds__(256) rotate_tiled_kernel(const __half *__restrict__ x,
                                                            const __half *__restrict__ suh,
                                                            unsigned char *__restrict__ xt, int m, int k)
@@ -219,10 +215,10 @@ __global__ void __launch_bounds__(256) rotate_tiled_kernel(const __half *__restr
         const float s = 0.08838834764831845f;
         __half2 o0 = __floats2half2_rn(v[0] * s, v[1] * s);
         __half2 o1 = __floats2half2_rn(v[2] * s, v[3] * s);
-        const int kb = c >> 5, chunk = (c & 31) >> 3, within = c & 7;
-        const int64_t tile = (int64_t)(r >> 7) * (k >> 5) + kb;
+        const int kb = c >> 6, chunk = (c & 63) >> 3, within = c & 7;
+        const int64_t tile = (int64_t)(r >> 7) * (k >> 6) + kb;
         const int row = r & 127;
-        unsigned char *dst = xt + tile * kATileBytes + row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4) + within * 2;
+        unsigned char *dst = xt + tile * kATileBytes + row * 128 + ((chunk ^ (row & 7)) << 4) + within * 2;
         uint2 out;
         out.x = *reinterpret_cast<uint32_t *>(&o0);
         out.y = *reinterpret_cast<uint32_t *>(&o1);
@@ -289,8 +285,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmParams 
     const int tm = blockIdx.x / tiles_n, tn = blockIdx.x - (blockIdx.x / tiles_n) * tiles_n;
     const int m0 = tm * kBM * kMT;
     const int kblocks = p.k / kBK;
-    // M tiles that hold any row (the rest would be all padding)
-    const int mt_count = (p.m - m0 + kBM - 1) / kBM < kMT ? (p.m - m0 + kBM - 1) / kBM : kMT;
+    const int mt_count = (p.m - m0) > kBM ? kMT : 1;  // skip an M tile that is all padding
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -359,11 +354,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmParams 
                 const uint32_t b0 = a0 + kMT * kATileBytes;
 #pragma unroll
                 for (int kk = 0; kk < kBK / 16; ++kk) {
-                    // B: atoms of 8 k rows (1024 B apart), 64-column groups (kBK/8 atoms apart)
-                    const uint64_t bdesc = smem_desc(b0 + kk * 2048, (kBK / 8) * 1024, 1024, kSw128);
+                    const uint64_t bdesc = smem_desc(b0 + kk * 2048, 8192, 1024);
                     for (int mt = 0; mt < mt_count; ++mt) {
-                        // A: 8-row groups 512 B apart; k16 = 32 bytes into the 64-byte row
-                        const uint64_t adesc = smem_desc(a0 + mt * kATileBytes + kk * 32, 16, 512, kSw64);
+                        const uint64_t adesc = smem_desc(a0 + mt * kATileBytes + kk * 32, 16, 1024);
                         mma_f16_ss(tmem + (uint32_t)(mt * kBN), adesc, bdesc, idesc, (kb | kk) ? 1u : 0u);
                     }
                 }
@@ -396,19 +389,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmParams 
             unsigned char *st = stages + s * kStage;
             unsigned char *bt = st + kMT * kATileBytes;
             const unsigned char *tr = bt + kBTileBytes;
-            // decoder warp dw takes tiles 4(dw/2) .. 4(dw/2)+3 and the rows of
-            // parity dw%2 (compile-time bit windows): lane l decodes row
-            // 2(l%8) + dw%2 of tile 4(dw/2) + l/8
-            static_assert((kBK / 16) * (kBN / 16) == 2 * kDecWarps, "tiles per stage");
+            // 4 tiles per warp; lane l decodes rows 2(l%8) and 2(l%8)+1 of tile
+            // l/8 (one parity per pass: compile-time bit windows)
+            static_assert((kBK / 16) * (kBN / 16) == 4 * kDecWarps, "tiles per stage");
             {
-                const int T = (dw >> 1) * 4 + (lane >> 3);
+                const int T = dw * 4 + (lane >> 3);
                 const int trow = T / (kBN / 16), tcol = T - (T / (kBN / 16)) * (kBN / 16);
                 const uint32_t *tw = reinterpret_cast<const uint32_t *>(tr + T * 32 * K);
                 const int r0 = 2 * (lane & 7);
-                if (dw & 1)
-                    decode_row_to_b<K, 1>(tw, r0 + 1, p.cb, bt, trow, tcol);
-                else
-                    decode_row_to_b<K, 0>(tw, r0, p.cb, bt, trow, tcol);
+                decode_row_to_b<K, 0>(tw, r0, p.cb, bt, trow, tcol);
+                decode_row_to_b<K, 1>(tw, r0 + 1, p.cb, bt, trow, tcol);
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -526,7 +516,7 @@ static exl3_status launch_gemm_t(const GemmParams &p, cudaStream_t stream)
 
 extern "C" size_t exl3_gemm_workspace_size(int64_t m, int64_t k, int64_t n, int K)
 {
-    if (m < 1 || k < 128 || n < 128 || (k % 128) || (n % 128) || K < 1 || K > 8)
+    if (m < 1 || k < 128 || n < 256 || (k % 128) || (n % 256) || K < 1 || K > 8)
         return 0;
     return 1024 + exl3::gemm_xt_bytes(m, k);
 }
