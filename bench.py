@@ -44,6 +44,10 @@ def parse():
     ap.add_argument("--no-gemm", action="store_true", help="skip the m=2048 GEMM line item")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--profile", default=None,
+                    help="profiling mode (no timing, no JSON): 'gemv-set' runs the decode GEMV set eagerly "
+                         "warmup+steps times; 'gemm' runs the m=2048 prefill GEMM warmup+steps times; "
+                         "'gemv-layer:k:n:K' runs one m=1 layer")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch without programmatic dependent launch (PDL is valid here: weights are immutable)")
     return ap.parse_args()
@@ -380,8 +384,44 @@ def bench_gemm(exl3, torch, peaks, stream):
             "peak_source": peaks["source"] + " bf16 cuBLAS burst (fp16 rate is the same)"}
 
 
+def run_profile(args):
+    """Launch-only mode for ncu: the same kernels as the timed run, no events."""
+    import torch
+
+    from trellis_coded_bit_b200 import exl3
+
+    exl3.load()
+    if not args.no_pdl:
+        exl3.exl3_set_launch_flags(exl3.EXL3_LAUNCH_PDL)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    what = args.profile
+    if what == "gemm":
+        m, k, n, K = 2048, 8192, 28672, 3
+        L = inputs.make_layer(m, k, n, K, inputs.seed_for(3, 2))
+        x, t, suh, svh = dev(L.x), dev(L.trellis), dev(L.suh), dev(L.svh)
+        ws = exl3.new_workspace(exl3.exl3_gemm_workspace_size(m, k, n, K))
+        for _ in range(args.warmup + args.steps):
+            exl3.exl3_gemm(x, t, suh, svh, K, workspace=ws)
+    else:
+        if what == "gemv-set":
+            layers = make_layers()
+        else:
+            _, k, n, K = what.split(":")
+            layers = [inputs.make_layer(1, int(k), int(n), int(K), seed=1)]
+        D = [dict(x=dev(L.x), t=dev(L.trellis), suh=dev(L.suh), svh=dev(L.svh), L=L,
+                  ws=exl3.new_workspace(exl3.exl3_gemv_workspace_size(L.m, L.k, L.n, L.K))) for L in layers]
+        for _ in range(args.warmup + args.steps):
+            for d in D:
+                exl3.exl3_gemv(d["x"], d["t"], d["suh"], d["svh"], d["L"].K, workspace=d["ws"])
+    torch.cuda.synchronize()
+    print("profile run done: %s" % what)
+
+
 def main():
     args = parse()
+    if args.profile:
+        run_profile(args)
+        return
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
