@@ -149,9 +149,19 @@ exl3_status exl3_gemv_noalloc(const void *x, const uint16_t *trellis, const void
  * exl3_gemm -- the linear layer on the tensor cores (tcgen05 / TMEM), any
  * m >= 1, tuned for m >= 64 ([GEMM] section GEMM内核: Hadamard rotation of the
  * input, then the dequantising matmul; the kernel map picks tiles by shape).
- * `workspace` (at least exl3_gemm_workspace_size bytes, zero-filled once after
- * allocation) holds the rotated activations x' (m x k fp16) and a status
- * word.  Same argument conventions as exl3_gemv.
+ * n must be a multiple of 256 (EXL3_ERR_UNSUPPORTED otherwise).  The kernel
+ * is persistent (one CTA per SM) and splits the work evenly over the CTAs by
+ * (256 x 256 output tile, 64-channel k block) units, so a tile can be shared
+ * by several CTAs; their fp32 partial sums meet in the workspace and are
+ * added in a fixed order, so results are deterministic.
+ * `workspace` (at least exl3_gemm_workspace_size bytes -- a size that depends
+ * on the current device's SM count, so query it on the device that runs the
+ * call -- zero-filled once after allocation) holds a status word, per-tile
+ * arrival counters (each call returns them to zero), the rotated activations
+ * x' (m rounded up to 256, x k fp16) and the split partial sums (two 256 KB
+ * slots per CTA).  Same argument conventions as exl3_gemv.  After a call
+ * that reported EXL3_ERR_TIMEOUT the counters may be left part-way: zero-fill
+ * the workspace again before its next use.
  */
 size_t exl3_gemm_workspace_size(int64_t m, int64_t k, int64_t n, int K);
 exl3_status exl3_gemm(const void *x, const uint16_t *trellis, const void *suh, const void *svh,

@@ -282,15 +282,34 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64
     return true;
 }
 
+// Bounded wait for a role that is not on the critical path at that moment (a
+// producer running ahead, an epilogue waiting out a whole k loop): it sleeps
+// between polls so that its waiting takes no issue slots from the warps doing
+// the work.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity, uint64_t limit_ns,
+                                                unsigned sleep_ns)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        __nanosleep(sleep_ns);
+        if (global_ns() - t0 > limit_ns)
+            return false;
+    }
+    return true;
+}
+
 // Warp-uniform bounded wait: lane 0 decides (so a timeout cannot split the
 // warp), then the other lanes observe the completed phase themselves, which
 // cannot move on before this warp releases the stage.
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns)
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns,
+                                          unsigned sleep_ns = 0)
 {
     const int lane = threadIdx.x & 31;
     bool ok = true;
     if (lane == 0)
-        ok = mbar_wait(bar, parity, limit_ns);
+        ok = sleep_ns ? mbar_wait_sleep(bar, parity, limit_ns, sleep_ns) : mbar_wait(bar, parity, limit_ns);
     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
     if (ok && lane != 0)
         mbar_wait(bar, parity, kDefaultWaitNs);

@@ -26,6 +26,9 @@ uint64_t wait_limit_ns();
 // Process-wide launch options (EXL3_LAUNCH_PDL).
 unsigned launch_flags();
 
+// Streaming multiprocessors of the current device (looked up once).
+int num_sms();
+
 // Launches `kernel` with the library's launch options: with EXL3_LAUNCH_PDL
 // the launch allows programmatic dependent launch (the kernel itself calls
 // griddepcontrol.wait before touching anything but weights).

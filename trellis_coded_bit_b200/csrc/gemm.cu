@@ -10,24 +10,40 @@
 //      it as fp16 directly in the tensor core's canonical K-major, 128-byte
 //      swizzled tile layout ([m/128][k/64] tiles of 128 rows x 64 channels,
 //      16 KB each), so one 1-D bulk copy moves one A tile into shared memory.
-//   2. The main kernel: one CTA per 256 x 256 output tile (two M=128 tiles
-//      that share every decoded B stage), 18 warps:
-//        warp 0   producer: per 64-channel k block, bulk-copies the two A
-//                 tiles and the 4 trellis tile rows (16 tiles each) into a
-//                 stage, completing on an mbarrier (no multicast);
-//        warp 1   allocates 512 TMEM columns; one lane issues
+//   2. The main kernel is persistent and "stream-K" balanced: the work units
+//      are (256 x 256 output tile, 64-channel k block) pairs in tile order,
+//      and CTA c of G (G <= one per SM) owns units [cU/G, (c+1)U/G), so every
+//      CTA gets the same work whatever the tile count (no last partial
+//      wave).  A CTA's range splits at tile boundaries into segments.  A
+//      segment that covers a whole tile is finished directly; one that covers
+//      part of a tile writes its fp32 accumulators to the workspace, and the
+//      last segment to arrive on the tile's counter (atomic ticket, no
+//      spinning) sums every segment's partials in segment order
+//      (deterministic) and finishes the tile.  23 warps:
+//        warp 0   A producer: bulk-copies the two A tiles of each unit into a
+//                 3-stage ring (no multicast; it sleeps between polls);
+//        warp 2   trellis producer: bulk-copies each unit's 4 trellis tile
+//                 rows (16 tiles each) into a ring as deep as the shared
+//                 memory left allows (12 stages at K = 1 .. 2 at K = 8),
+//                 so the decoders never wait for HBM (sleeps between polls);
+//        warp 1   allocates 512 TMEM columns (two 128 x 256 fp32
+//                 accumulators); one lane issues
 //                 tcgen05.mma.cta_group::1.kind::f16 (M=128, N=256, K=16,
-//                 fp32 accumulate, A K-major, B MN-major) and commits to
-//                 mbarriers that free the stage / signal the epilogue;
-//        warps 2..17 decode: lane u of a warp decodes run u (8 consecutive
-//                 output channels of one input channel) of one trellis tile,
-//                 sums the codebook halves in fp16 (RNE, the exact W_hat) and
-//                 stores the 16-byte run into the MN-major 128-byte-swizzled
-//                 B stage; fence.proxy.async then an mbarrier arrive.
-//      After the k loop, warps 2..5 (one TMEM lane quarter each) read the
-//      accumulators with tcgen05.ld, apply the 128-point output rotation as
-//      H4 (x) H32 (32-point butterflies in registers, a TMEM round trip, then
-//      the 4-point stage), scale by svh/sqrt(128) and store fp16 y.
+//                 A K-major, B MN-major) and commits to mbarriers that free
+//                 the A and B stages and, at a segment end, hand the
+//                 accumulators to the epilogue;
+//        warps 3..18 decode: lane u of a warp decodes two rows of one trellis
+//                 tile, sums the codebook halves in fp16 (RNE, the exact
+//                 W_hat) and stores them into the MN-major 128-byte-swizzled
+//                 B stage (3-stage ring); fence.proxy.async, mbarrier arrive;
+//        warps 19..22 epilogue (one TMEM lane quarter each): tcgen05.ld of the
+//                 accumulators, the 128-point output rotation as
+//                 H4 (x) H32 (32-point butterflies in registers, a TMEM round
+//                 trip, then the 4-point stage), svh/sqrt(128), fp16 y; or the
+//                 partial-sum write and the ticket.
+//   Shared memory is addressed from the dynamic shared array (the 1024-byte
+//   alignment the swizzled tiles need is an offset, not an integer cast), so
+//   the decoders' loads and stores stay shared-space instructions.
 //   All waits are bounded; a timeout is recorded in the workspace status word
 //   and every role drains its in-flight copies / MMAs before the CTA exits.
 #include <cuda_fp16.h>
@@ -39,33 +55,47 @@ namespace exl3 {
 
 constexpr int kBM = 128;             // rows per MMA tile (TMEM lanes)
 constexpr int kMT = 2;               // M tiles per CTA sharing one decoded B
-constexpr int kBN = 256;             // output channels per CTA (MMA N)
-constexpr int kBK = 64;              // input channels per stage
+constexpr int kBN = 256;             // output channels per tile (MMA N)
+constexpr int kBK = 64;              // input channels per unit
 constexpr int kDecWarps = 16;
-constexpr int kGemmThreads = 32 * (2 + kDecWarps);
-constexpr int kATileBytes = kBM * kBK * 2;   // 16 KB
-constexpr int kBTileBytes = kBK * kBN * 2;   // 32 KB
-constexpr int kTmemCols = kMT * kBN;         // 512
+// 23 warps: the decoders carry no epilogue state, and the epilogue warps do
+// not hold up decoding while they drain the accumulators
+constexpr int kWarpProducerA = 0, kWarpMma = 1, kWarpProducerT = 2, kWarpDec0 = 3;
+constexpr int kWarpEpi0 = kWarpDec0 + kDecWarps;                   // 19..22
+constexpr int kGemmThreads = 32 * (kWarpEpi0 + 4);                 // 736
+constexpr int kATileBytes = kBM * kBK * 2;                  // 16 KB
+constexpr int kAStageBytes = kMT * kATileBytes;             // 32 KB
+constexpr int kBStageBytes = kBK * kBN * 2;                 // 32 KB
+constexpr int kAStages = 3;
+constexpr int kBStages = 3;
+constexpr int kMaxTStages = 12;
+constexpr int kTmemCols = kMT * kBN;                        // 512
+constexpr int kPartialFloats = kMT * kBM * kBN;             // one split segment: 256 KB
 
 __host__ __device__ constexpr int gemm_trellis_stage_bytes(int K)
 {
     return (kBK / 16) * (kBN / 16) * 32 * K;  // 4 tile rows x 16 tiles
 }
 
-__host__ __device__ constexpr int gemm_stage_bytes(int K)
-{
-    return kMT * kATileBytes + kBTileBytes + ((gemm_trellis_stage_bytes(K) + 1023) & ~1023);
-}
+// Trellis ring depth: whatever shared memory the A and B rings leave (up to
+// 227 KB per CTA), at most kMaxTStages stages.
+constexpr int kSmemLimit = 232448;
+constexpr int kTBudget = kSmemLimit - 2048 - kAStages * kAStageBytes - kBStages * kBStageBytes;
 
-__host__ __device__ constexpr int gemm_stages(int K)
+__host__ __device__ constexpr int gemm_t_stages(int K)
 {
-    return (220 * 1024) / gemm_stage_bytes(K) >= 3 ? 3 : 2;
+    return kTBudget / gemm_trellis_stage_bytes(K) > kMaxTStages ? kMaxTStages
+                                                               : kTBudget / gemm_trellis_stage_bytes(K);
 }
 
 __host__ __device__ constexpr int gemm_smem_bytes(int K)
 {
-    return 1024 /* alignment slack */ + 1024 /* barriers etc. */ + gemm_stages(K) * gemm_stage_bytes(K);
+    return 1024 /* alignment slack */ + 1024 /* barriers */ + kAStages * kAStageBytes +
+           kBStages * kBStageBytes + gemm_t_stages(K) * gemm_trellis_stage_bytes(K);
 }
+
+static_assert(gemm_t_stages(8) >= 2 && gemm_smem_bytes(8) <= kSmemLimit && gemm_smem_bytes(1) <= kSmemLimit,
+              "shared memory per CTA");
 
 // ----------------------------------------------------- tcgen05 wrappers ---
 
@@ -116,16 +146,6 @@ __device__ __forceinline__ void fence_proxy_async_smem()
     asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
 }
 
-#define EXL3_TMEM_LD32(taddr, v)                                                                          \
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14," \
-                 "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"          \
-                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),     \
-                   "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), \
-                   "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),           \
-                   "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),           \
-                   "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])            \
-                 : "r"(taddr))
-
 #define EXL3_TMEM_ST32(taddr, v)                                                                          \
     asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13," \
                  "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n" ::"r"(   \
@@ -137,22 +157,36 @@ __device__ __forceinline__ void fence_proxy_async_smem()
                  "r"(v[29]), "r"(v[30]), "r"(v[31])                                                        \
                  : "memory")
 
-#define EXL3_TMEM_LD8(taddr, v)                                                                           \
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"                \
-                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),     \
-                   "=r"(v[7])                                                                              \
-                 : "r"(taddr))
+// A TMEM load and its wait in one statement: PTX leaves the destination
+// registers of tcgen05.ld undefined until tcgen05.wait::ld, so the compiler
+// must not be able to touch them (a spill, say) in between.
+#define EXL3_TMEM_LD32(taddr, v)                                                                          \
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14," \
+                 "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"          \
+                 "tcgen05.wait::ld.sync.aligned;\n"                                                       \
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), \
+                   "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), \
+                   "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), \
+                   "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), \
+                   "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), \
+                   "=r"(v[31]) \
+                 : "r"(taddr)                                                                              \
+                 : "memory")
 
-// Wait for tcgen05.ld to land; the 32 destination registers are tied to the
-// wait so that no use of them can be scheduled before it.
-#define EXL3_TMEM_WAIT_LD32(v)                                                                            \
-    asm volatile("tcgen05.wait::ld.sync.aligned;\n"                                                       \
-                 : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]),     \
-                   "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]), "+r"(v[12]), "+r"(v[13]), \
-                   "+r"(v[14]), "+r"(v[15]), "+r"(v[16]), "+r"(v[17]), "+r"(v[18]), "+r"(v[19]),           \
-                   "+r"(v[20]), "+r"(v[21]), "+r"(v[22]), "+r"(v[23]), "+r"(v[24]), "+r"(v[25]),           \
-                   "+r"(v[26]), "+r"(v[27]), "+r"(v[28]), "+r"(v[29]), "+r"(v[30]), "+r"(v[31])            \
-                 :                                                                                         \
+// Four 8-column loads at taddr, taddr + 32, + 64, + 96 into v[0..31], then the wait.
+#define EXL3_TMEM_LD8X4(taddr, v)                                                                         \
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%32];\n"               \
+                 "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%8,%9,%10,%11,%12,%13,%14,%15}, [%33];\n"         \
+                 "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%16,%17,%18,%19,%20,%21,%22,%23}, [%34];\n"       \
+                 "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%24,%25,%26,%27,%28,%29,%30,%31}, [%35];\n"       \
+                 "tcgen05.wait::ld.sync.aligned;\n"                                                       \
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), \
+                   "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), \
+                   "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), \
+                   "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), \
+                   "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), \
+                   "=r"(v[31]) \
+                 : "r"(taddr), "r"((taddr) + 32u), "r"((taddr) + 64u), "r"((taddr) + 96u)                  \
                  : "memory")
 
 __device__ __forceinline__ void tmem_wait_st()
@@ -256,236 +290,444 @@ struct GemmParams {
     const uint16_t *trellis;
     const __half *svh;
     __half *y;
-    int m, k, n;
+    float *partials;           // [2 G][kPartialFloats] split-segment accumulators
+    uint32_t *counters;        // [tiles] arrival tickets (return to zero)
     uint32_t *status;
+    int m, k, n;
+    int tiles_n;               // n / 256
+    int kb_count;              // k / 64 units per tile
+    uint32_t units;            // tiles * kb_count (units * ctas < 2^32)
+    int ctas;                  // grid size G
     uint64_t wait_ns;
     Codebook cb;
 };
 
+struct GemmBars {
+    uint64_t afull[kAStages], aempty[kAStages];
+    uint64_t bfull[kBStages], bempty[kBStages];
+    uint64_t tfull[kMaxTStages], tempty[kMaxTStages];
+    uint64_t acc_full, acc_empty, drain;
+    uint32_t tmem_slot;
+    int abort;
+    int ticket;
+};
+static_assert(sizeof(GemmBars) <= 1024, "barrier block");
+
+// CTA owning unit u: the largest c with floor(c U / G) <= u.  (32-bit: the
+// host guarantees U * G < 2^32.)
+__device__ __forceinline__ int gemm_owner(uint32_t u, uint32_t U, uint32_t G)
+{
+    return (int)(((u + 1) * G - 1) / U);
+}
+
+// Partial-sum slot of CTA c's segment in the tile starting at unit tb: its
+// first segment (the one holding its first unit) uses slot 2c, its last 2c+1.
+__device__ __forceinline__ int gemm_slot(uint32_t c, uint32_t tb, uint32_t U, uint32_t G)
+{
+    return (int)((c * U / G >= tb) ? 2 * c : 2 * c + 1);
+}
+
+// Named barrier over the four epilogue warps.
+__device__ __forceinline__ void epi_sync()
+{
+    asm volatile("bar.sync 1, 128;\n" ::: "memory");
+}
+
+// Epilogue of one segment [u, se) (units of one tile), run by the four
+// epilogue warps (one TMEM lane quarter each): waits for the accumulators, then either finishes the tile (output
+// rotation, svh, fp16 y) or writes the segment's partial sums and takes a
+// ticket -- the last segment of the tile to arrive sums all partials and
+// finishes it.  Releases the accumulators to the MMA issuer at the end.
+// Returns false if the wait ran out (the caller stops).
+__device__ __forceinline__ bool gemm_epilogue(const GemmParams &p, GemmBars &bars, uint32_t tmem, int seg,
+                                              uint32_t u, uint32_t se, uint32_t U, uint32_t G, uint32_t KB)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int quarter = warp & 3;  // TMEM lanes this warp may access
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const int erow = quarter * 32 + lane;  // row within an M tile
+    float4 *const parts = reinterpret_cast<float4 *>(p.partials);
+    volatile int *abort_flag = &bars.abort;
+    const uint32_t t = u / KB;
+    const uint32_t tb = t * KB, te = tb + KB;
+    const bool whole = u == tb && se == te;
+    const int tm = (int)(t / p.tiles_n), tn = (int)(t - (t / p.tiles_n) * p.tiles_n);
+    const int mt_count = (p.m - tm * kBM * kMT) > kBM ? kMT : 1;
+    if (!warp_wait(&bars.acc_full, (uint32_t)seg & 1u, p.wait_ns)) {
+        if (lane == 0) {
+            record_timeout(p.status);
+            *abort_flag = 1;
+        }
+        return false;
+    }
+    tc_fence_after();
+    if (*abort_flag)
+        return false;
+    int nseg = 1, c_lo = 0;
+    bool finish = true;
+    if (!whole) {
+        // this segment's fp32 accumulators -> its slot, 16-byte chunk
+        // (mt, 4-column group g, row): consecutive lanes, consecutive chunks
+        c_lo = gemm_owner(tb, U, G);
+        nseg = gemm_owner(te - 1, U, G) - c_lo + 1;
+        float4 *slot = parts + (size_t)gemm_slot(blockIdx.x, tb, U, G) * (kPartialFloats / 4);
+        for (int mt = 0; mt < mt_count; ++mt) {
+#pragma unroll 1
+            for (int cc = 0; cc < kBN / 32; ++cc) {
+                uint32_t r[32];
+                EXL3_TMEM_LD32(tmem + lane_base + (uint32_t)(mt * kBN + 32 * cc), r);
+#pragma unroll
+                for (int g = 0; g < 8; ++g)
+                    __stcg(slot + ((mt * 64 + cc * 8 + g) * kBM + erow),
+                           make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]),
+                                       __uint_as_float(r[4 * g + 2]), __uint_as_float(r[4 * g + 3])));
+            }
+        }
+        __threadfence();
+        epi_sync();
+        if (warp == kWarpEpi0 && lane == 0) {
+            const uint32_t prev = atomicAdd(&p.counters[t], 1u);
+            const int last = prev == (uint32_t)(nseg - 1) ? 1 : 0;
+            if (last) {
+                __threadfence();
+                p.counters[t] = 0u;  // every segment has arrived: re-arm for the next call
+            }
+            bars.ticket = last;
+        }
+        epi_sync();
+        finish = bars.ticket != 0;
+    }
+    if (finish && !whole) {
+        // every segment's partials, summed in segment order, accumulated in
+        // TMEM (s = p0; s += p1; ...): 32 columns (8 loads in flight) a step
+        for (int mt = 0; mt < mt_count; ++mt) {
+#pragma unroll 1
+            for (int j = 0; j < nseg; ++j) {
+                const float4 *src = parts + (size_t)gemm_slot((uint32_t)(c_lo + j), tb, U, G) * (kPartialFloats / 4) +
+                                    (mt * 64 * kBM + erow);
+#pragma unroll 1
+                for (int cc = 0; cc < kBN / 32; ++cc) {
+                    float4 q[8];
+#pragma unroll
+                    for (int g = 0; g < 8; ++g)
+                        q[g] = __ldcg(src + (cc * 8 + g) * kBM);
+                    const uint32_t ta = tmem + lane_base + (uint32_t)(mt * kBN + 32 * cc);
+                    uint32_t r[32];
+                    if (j == 0) {
+#pragma unroll
+                        for (int g = 0; g < 8; ++g) {
+                            r[4 * g] = __float_as_uint(q[g].x);
+                            r[4 * g + 1] = __float_as_uint(q[g].y);
+                            r[4 * g + 2] = __float_as_uint(q[g].z);
+                            r[4 * g + 3] = __float_as_uint(q[g].w);
+                        }
+                    } else {
+                        EXL3_TMEM_LD32(ta, r);
+#pragma unroll
+                        for (int g = 0; g < 8; ++g) {
+                            r[4 * g] = __float_as_uint(__uint_as_float(r[4 * g]) + q[g].x);
+                            r[4 * g + 1] = __float_as_uint(__uint_as_float(r[4 * g + 1]) + q[g].y);
+                            r[4 * g + 2] = __float_as_uint(__uint_as_float(r[4 * g + 2]) + q[g].z);
+                            r[4 * g + 3] = __float_as_uint(__uint_as_float(r[4 * g + 3]) + q[g].w);
+                        }
+                    }
+                    EXL3_TMEM_ST32(ta, r);
+                }
+                tmem_wait_st();
+            }
+        }
+    }
+    if (finish) {
+        for (int mt = 0; mt < mt_count; ++mt) {
+            const int row = tm * kBM * kMT + mt * kBM + erow;
+            for (int hb = 0; hb < kBN / 128; ++hb) {
+                const uint32_t col0 = (uint32_t)(mt * kBN + hb * 128);
+                // 32-point butterflies on each 32-column chunk, written back to TMEM
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t r[32];
+                    EXL3_TMEM_LD32(tmem + lane_base + col0 + 32 * c, r);
+                    float v[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        v[i] = __uint_as_float(r[i]);
+                    fwht32(v);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        r[i] = __float_as_uint(v[i]);
+                    EXL3_TMEM_ST32(tmem + lane_base + col0 + 32 * c, r);
+                    tmem_wait_st();
+                }
+                // 4-point stage across the chunks, scale, fp16, store
+#pragma unroll 1
+                for (int o = 0; o < 4; ++o) {
+                    uint32_t w[32];  // [chunk c][8 columns]
+                    EXL3_TMEM_LD8X4(tmem + lane_base + col0 + 8 * o, w);
+                    if (row < p.m) {
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            const int ncol = tn * kBN + hb * 128 + 32 * c + 8 * o;
+                            const uint4 sv4 = *reinterpret_cast<const uint4 *>(p.svh + ncol);
+                            const __half2 *sv = reinterpret_cast<const __half2 *>(&sv4);
+                            uint32_t pk[4];
+#pragma unroll
+                            for (int e = 0; e < 8; e += 2) {
+                                float z[2];
+#pragma unroll
+                                for (int d = 0; d < 2; ++d) {
+                                    const float a0 = __uint_as_float(w[0 + e + d]);
+                                    const float a1 = __uint_as_float(w[8 + e + d]);
+                                    const float a2 = __uint_as_float(w[16 + e + d]);
+                                    const float a3 = __uint_as_float(w[24 + e + d]);
+                                    const float s01 = a0 + a1, d01 = a0 - a1, s23 = a2 + a3,
+                                                d23 = a2 - a3;
+                                    // H4 row c: c=0 (+,+,+,+) c=1 (+,-,+,-) c=2 (+,+,-,-) c=3 (+,-,-,+)
+                                    z[d] = c == 0 ? s01 + s23 : c == 1 ? d01 + d23 : c == 2 ? s01 - s23 : d01 - d23;
+                                }
+                                const float sc = 0.08838834764831845f;
+                                __half2 h = __floats2half2_rn(z[0] * sc * __low2float(sv[e >> 1]),
+                                                              z[1] * sc * __high2float(sv[e >> 1]));
+                                pk[e >> 1] = *reinterpret_cast<uint32_t *>(&h);
+                            }
+                            *reinterpret_cast<uint4 *>(p.y + (int64_t)row * p.n + ncol) =
+                                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        }
+                    }
+                }
+            }
+        }
+    }
+    // hand the accumulators back to the MMA issuer
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0)
+        mbar_arrive(&bars.acc_empty);
+    return true;
+}
+
+
 template <int K>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmParams p)
 {
-    constexpr int S = gemm_stages(K);
-    constexpr int kStage = gemm_stage_bytes(K);
-    constexpr int kTrellisBytes = gemm_trellis_stage_bytes(K);
+    constexpr int TS = gemm_t_stages(K);
+    constexpr int kTrBytes = gemm_trellis_stage_bytes(K);
     constexpr int kTileRowBytes = (kBN / 16) * 32 * K;
-    extern __shared__ unsigned char smem_raw[];
-    unsigned char *smem = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint64_t *full_a = reinterpret_cast<uint64_t *>(smem);  // A + trellis landed
-    uint64_t *full_b = full_a + S;                            // B decoded
-    uint64_t *empty = full_b + S;                             // MMAs done with the stage
-    uint64_t *acc_full = empty + S;
-    uint64_t *drain = acc_full + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    unsigned char *stages = smem + 1024;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+    GemmBars &bars = *reinterpret_cast<GemmBars *>(smem);
+    unsigned char *aring = smem + 1024;
+    unsigned char *bring = aring + kAStages * kAStageBytes;
+    unsigned char *tring = bring + kBStages * kBStageBytes;
+    volatile int *abort_flag = &bars.abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tiles_n = p.n / kBN;
-    const int tm = blockIdx.x / tiles_n, tn = blockIdx.x - (blockIdx.x / tiles_n) * tiles_n;
-    const int m0 = tm * kBM * kMT;
-    const int kblocks = p.k / kBK;
-    const int mt_count = (p.m - m0) > kBM ? kMT : 1;  // skip an M tile that is all padding
+    const uint32_t U = p.units;
+    const uint32_t G = (uint32_t)p.ctas;
+    const uint32_t u0 = blockIdx.x * U / G, u1 = (blockIdx.x + 1) * U / G;
+    const int nu = (int)(u1 - u0);
+    const uint32_t KB = (uint32_t)p.kb_count;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&full_a[s], 1);
-            mbar_init(&full_b[s], kDecWarps);
-            mbar_init(&empty[s], 1);
+        for (int s = 0; s < kAStages; ++s) {
+            mbar_init(&bars.afull[s], 1);
+            mbar_init(&bars.aempty[s], 1);
         }
-        mbar_init(acc_full, 1);
-        mbar_init(drain, 1);
-        *abort_flag = 0;
+        for (int s = 0; s < kBStages; ++s) {
+            mbar_init(&bars.bfull[s], kDecWarps);
+            mbar_init(&bars.bempty[s], 1);
+        }
+        for (int s = 0; s < TS; ++s) {
+            mbar_init(&bars.tfull[s], 1);
+            mbar_init(&bars.tempty[s], kDecWarps);
+        }
+        mbar_init(&bars.acc_full, 1);
+        mbar_init(&bars.acc_empty, 4);
+        mbar_init(&bars.drain, 1);
+        bars.abort = 0;
+        bars.ticket = 0;
         fence_mbar_init();
     }
-    if (warp == 1)
-        tmem_alloc(tmem_slot, kTmemCols);
+    if (warp == kWarpMma)
+        tmem_alloc(&bars.tmem_slot, kTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    grid_dep_wait();  // x' comes from the rotation kernel just before
+    const uint32_t tmem = bars.tmem_slot;
+    // weights (trellis) may stream at once; everything else waits for the
+    // preceding kernel (x' comes from the rotation kernel just before)
+    if (warp != kWarpProducerT)
+        grid_dep_wait();
 
-    if (warp == 0) {
-        // ------------------------------------------------------ producer ---
+    if (warp == kWarpProducerA) {
+        // ---------------------------------------------------- A producer ---
         if (lane == 0) {
+            uint32_t t = u0 / KB;
+            int kb = (int)(u0 - t * KB);
+            int tm = (int)(t / p.tiles_n);
+            int mt_count = (p.m - tm * kBM * kMT) > kBM ? kMT : 1;  // skip an all-padding M tile
             int issued = 0;
-            for (int kb = 0; kb < kblocks; ++kb) {
-                const int s = kb % S;
-                const uint32_t ph = (uint32_t)(kb / S) & 1u;
-                if (!mbar_wait(&empty[s], ph ^ 1u, p.wait_ns)) {
+            for (int i = 0; i < nu; ++i) {
+                const int s = i % kAStages;
+                if (!mbar_wait_sleep(&bars.aempty[s], ((uint32_t)(i / kAStages) & 1u) ^ 1u, p.wait_ns, 100)) {
                     record_timeout(p.status);
                     *abort_flag = 1;
                     break;
                 }
-                unsigned char *st = stages + s * kStage;
-                mbar_arrive_expect_tx(&full_a[s], (uint32_t)(mt_count * kATileBytes + kTrellisBytes));
+                unsigned char *dst = aring + s * kAStageBytes;
+                mbar_arrive_expect_tx(&bars.afull[s], (uint32_t)(mt_count * kATileBytes));
                 for (int mt = 0; mt < mt_count; ++mt) {
-                    const int64_t tile = (int64_t)((m0 >> 7) + mt) * kblocks + kb;
-                    bulk_g2s(st + mt * kATileBytes, p.xt + tile * kATileBytes, kATileBytes, &full_a[s]);
+                    const int64_t tile = (int64_t)(tm * kMT + mt) * (p.k / kBK) + kb;
+                    bulk_g2s(dst + mt * kATileBytes, p.xt + tile * kATileBytes, kATileBytes, &bars.afull[s]);
                 }
-                unsigned char *tr = st + kMT * kATileBytes + kBTileBytes;
-                for (int r = 0; r < kBK / 16; ++r) {
-                    const int64_t row = (int64_t)kb * (kBK / 16) + r;
-                    const uint16_t *src = p.trellis + (row * (p.n / 16) + (int64_t)tn * (kBN / 16)) * 16 * K;
-                    bulk_g2s(tr + r * kTileRowBytes, src, kTileRowBytes, &full_a[s]);
+                issued = i + 1;
+                if (++kb == (int)KB) {
+                    kb = 0;
+                    ++t;
+                    tm = (int)(t / p.tiles_n);
+                    mt_count = (p.m - tm * kBM * kMT) > kBM ? kMT : 1;
                 }
-                issued = kb + 1;
             }
-            for (int kb = (issued > S ? issued - S : 0); kb < issued; ++kb)
-                if (!mbar_wait(&full_a[kb % S], (uint32_t)(kb / S) & 1u, kDefaultWaitNs))
+            for (int i = (issued > kAStages ? issued - kAStages : 0); i < issued; ++i)
+                if (!mbar_wait(&bars.afull[i % kAStages], (uint32_t)(i / kAStages) & 1u, kDefaultWaitNs))
                     record_timeout(p.status);
         }
-    } else if (warp == 1) {
+    } else if (warp == kWarpProducerT) {
+        // ---------------------------------------------- trellis producer ---
+        if (lane == 0) {
+            uint32_t t = u0 / KB;
+            int kb = (int)(u0 - t * KB);
+            int tn = (int)(t % p.tiles_n);
+            const int64_t row_words = (int64_t)(p.n / 16) * 16 * K;  // one tile row of the matrix
+            int issued = 0;
+            for (int i = 0; i < nu; ++i) {
+                const int s = i % TS;
+                if (!mbar_wait_sleep(&bars.tempty[s], ((uint32_t)(i / TS) & 1u) ^ 1u, p.wait_ns, 200)) {
+                    record_timeout(p.status);
+                    *abort_flag = 1;
+                    break;
+                }
+                unsigned char *dst = tring + s * kTrBytes;
+                mbar_arrive_expect_tx(&bars.tfull[s], (uint32_t)kTrBytes);
+                const uint16_t *src = p.trellis + (int64_t)kb * (kBK / 16) * row_words + (int64_t)tn * 16 * 16 * K;
+#pragma unroll
+                for (int r = 0; r < kBK / 16; ++r)
+                    bulk_g2s(dst + r * kTileRowBytes, src + r * row_words, kTileRowBytes, &bars.tfull[s]);
+                issued = i + 1;
+                if (++kb == (int)KB) {
+                    kb = 0;
+                    ++t;
+                    tn = (int)(t % p.tiles_n);
+                }
+            }
+            for (int i = (issued > TS ? issued - TS : 0); i < issued; ++i)
+                if (!mbar_wait(&bars.tfull[i % TS], (uint32_t)(i / TS) & 1u, kDefaultWaitNs))
+                    record_timeout(p.status);
+        }
+    } else if (warp == kWarpMma) {
         // ----------------------------------------------------- MMA issuer ---
         if (lane == 0) {
             const uint32_t idesc = gemm_idesc();
+            uint32_t t = u0 / KB;
+            int kb = (int)(u0 - t * KB);
+            int mt_count = (p.m - (int)(t / p.tiles_n) * kBM * kMT) > kBM ? kMT : 1;
+            int seg = 0;
             bool ok = true;
-            int kb = 0;
-            for (; kb < kblocks; ++kb) {
-                const int s = kb % S;
-                const uint32_t ph = (uint32_t)(kb / S) & 1u;
-                if (!mbar_wait(&full_a[s], ph, p.wait_ns) || !mbar_wait(&full_b[s], ph, p.wait_ns)) {
+            for (int i = 0; i < nu; ++i) {
+                const bool seg_start = i == 0 || kb == 0;
+                const bool seg_end = i == nu - 1 || kb == (int)KB - 1;
+                if (seg_start && seg > 0) {
+                    // the epilogue has read (and released) the previous accumulators
+                    if (!mbar_wait(&bars.acc_empty, (uint32_t)(seg - 1) & 1u, p.wait_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                }
+                const int sa = i % kAStages, sb = i % kBStages;
+                if (!mbar_wait(&bars.afull[sa], (uint32_t)(i / kAStages) & 1u, p.wait_ns) ||
+                    !mbar_wait(&bars.bfull[sb], (uint32_t)(i / kBStages) & 1u, p.wait_ns)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t a0 = smem_addr(stages + s * kStage);
-                const uint32_t b0 = a0 + kMT * kATileBytes;
+                const uint32_t a0 = smem_addr(aring + sa * kAStageBytes);
+                const uint32_t b0 = smem_addr(bring + sb * kBStageBytes);
 #pragma unroll
                 for (int kk = 0; kk < kBK / 16; ++kk) {
                     const uint64_t bdesc = smem_desc(b0 + kk * 2048, 8192, 1024);
                     for (int mt = 0; mt < mt_count; ++mt) {
                         const uint64_t adesc = smem_desc(a0 + mt * kATileBytes + kk * 32, 16, 1024);
-                        mma_f16_ss(tmem + (uint32_t)(mt * kBN), adesc, bdesc, idesc, (kb | kk) ? 1u : 0u);
+                        mma_f16_ss(tmem + (uint32_t)(mt * kBN), adesc, bdesc, idesc,
+                                   (!seg_start || kk) ? 1u : 0u);
                     }
                 }
-                mma_commit(&empty[s]);
+                mma_commit(&bars.aempty[sa]);
+                mma_commit(&bars.bempty[sb]);
+                if (seg_end) {
+                    mma_commit(&bars.acc_full);
+                    ++seg;
+                }
+                if (++kb == (int)KB) {
+                    kb = 0;
+                    ++t;
+                    mt_count = (p.m - (int)(t / p.tiles_n) * kBM * kMT) > kBM ? kMT : 1;
+                }
             }
-            if (ok) {
-                mma_commit(acc_full);
-            } else {
+            if (!ok) {
                 record_timeout(p.status);
                 *abort_flag = 1;
             }
             // make sure no MMA is still writing TMEM when the CTA tears down
-            mma_commit(drain);
-            if (!mbar_wait(drain, 0, kDefaultWaitNs))
+            mma_commit(&bars.drain);
+            if (!mbar_wait(&bars.drain, 0, kDefaultWaitNs))
                 record_timeout(p.status);
         }
-    } else {
+    } else if (warp >= kWarpEpi0 && warp < kWarpEpi0 + 4) {
+        // ---------------------------------------------- epilogue warps ---
+        uint32_t seg_u = u0;
+        for (int seg = 0; seg_u < u1; ++seg) {
+            const uint32_t te = (seg_u / KB + 1) * KB;
+            const uint32_t seg_e = te < u1 ? te : u1;
+            if (!gemm_epilogue(p, bars, tmem, seg, seg_u, seg_e, U, G, KB))
+                break;
+            seg_u = seg_e;
+        }
+    } else if (warp >= kWarpDec0 && warp < kWarpDec0 + kDecWarps) {
         // ------------------------------------------------------- decoders ---
-        const int dw = warp - 2;
-        for (int kb = 0; kb < kblocks; ++kb) {
-            const int s = kb % S;
-            const uint32_t ph = (uint32_t)(kb / S) & 1u;
-            if (!warp_wait(&full_a[s], ph, p.wait_ns)) {
+        // 4 tiles per warp; lane l decodes rows 2(l%8) and 2(l%8)+1 of tile
+        // l/8 (one parity per call: compile-time bit windows)
+        static_assert((kBK / 16) * (kBN / 16) == 4 * kDecWarps, "tiles per unit");
+        const int dw = warp - kWarpDec0;
+        const int T = dw * 4 + (lane >> 3);
+        const int trow = T / (kBN / 16), tcol = T - (T / (kBN / 16)) * (kBN / 16);
+        const int toff = trow * kTileRowBytes + tcol * 32 * K;
+        const int r0 = 2 * (lane & 7);
+        for (int i = 0; i < nu; ++i) {
+            const int st = i % TS, sb = i % kBStages;
+            if (!warp_wait(&bars.tfull[st], (uint32_t)(i / TS) & 1u, p.wait_ns) ||
+                !warp_wait(&bars.bempty[sb], ((uint32_t)(i / kBStages) & 1u) ^ 1u, p.wait_ns)) {
                 if (lane == 0) {
                     record_timeout(p.status);
                     *abort_flag = 1;
                 }
                 break;
             }
-            unsigned char *st = stages + s * kStage;
-            unsigned char *bt = st + kMT * kATileBytes;
-            const unsigned char *tr = bt + kBTileBytes;
-            // 4 tiles per warp; lane l decodes rows 2(l%8) and 2(l%8)+1 of tile
-            // l/8 (one parity per pass: compile-time bit windows)
-            static_assert((kBK / 16) * (kBN / 16) == 4 * kDecWarps, "tiles per stage");
-            {
-                const int T = dw * 4 + (lane >> 3);
-                const int trow = T / (kBN / 16), tcol = T - (T / (kBN / 16)) * (kBN / 16);
-                const uint32_t *tw = reinterpret_cast<const uint32_t *>(tr + T * 32 * K);
-                const int r0 = 2 * (lane & 7);
-                decode_row_to_b<K, 0>(tw, r0, p.cb, bt, trow, tcol);
-                decode_row_to_b<K, 1>(tw, r0 + 1, p.cb, bt, trow, tcol);
-            }
+            const uint32_t *tw = reinterpret_cast<const uint32_t *>(tring + st * kTrBytes + toff);
+            unsigned char *bt = bring + sb * kBStageBytes;
+            decode_row_to_b<K, 0>(tw, r0, p.cb, bt, trow, tcol);
+            decode_row_to_b<K, 1>(tw, r0 + 1, p.cb, bt, trow, tcol);
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&full_b[s]);
-        }
-
-        // ------------------------------------------------------ epilogue ---
-        if (dw < 4) {
-            const int quarter = warp & 3;  // TMEM lanes this warp may access
-            const bool have = warp_wait(acc_full, 0, p.wait_ns);
-            if (!have) {
-                if (lane == 0)
-                    record_timeout(p.status);
-            } else if (!*abort_flag) {
-                tc_fence_after();
-                const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-                for (int mt = 0; mt < mt_count; ++mt) {
-                    const int row = m0 + mt * kBM + quarter * 32 + lane;
-                    for (int hb = 0; hb < kBN / 128; ++hb) {
-                        const uint32_t col0 = (uint32_t)(mt * kBN + hb * 128);
-                        // 32-point butterflies on each 32-column chunk, written back to TMEM
-#pragma unroll 1
-                        for (int c = 0; c < 4; ++c) {
-                            uint32_t r[32];
-                            EXL3_TMEM_LD32(tmem + lane_base + col0 + 32 * c, r);
-                            EXL3_TMEM_WAIT_LD32(r);
-                            float v[32];
-#pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                v[i] = __uint_as_float(r[i]);
-                            fwht32(v);
-#pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                r[i] = __float_as_uint(v[i]);
-                            EXL3_TMEM_ST32(tmem + lane_base + col0 + 32 * c, r);
-                            tmem_wait_st();
-                        }
-                        // 4-point stage across the chunks, scale, fp16, store
-#pragma unroll 1
-                        for (int o = 0; o < 4; ++o) {
-                            uint32_t u[32];  // [chunk c][8 columns]
-                            EXL3_TMEM_LD8(tmem + lane_base + col0 + 0 + 8 * o, (u + 0));
-                            EXL3_TMEM_LD8(tmem + lane_base + col0 + 32 + 8 * o, (u + 8));
-                            EXL3_TMEM_LD8(tmem + lane_base + col0 + 64 + 8 * o, (u + 16));
-                            EXL3_TMEM_LD8(tmem + lane_base + col0 + 96 + 8 * o, (u + 24));
-                            EXL3_TMEM_WAIT_LD32(u);
-                            if (row < p.m) {
-#pragma unroll
-                                for (int c = 0; c < 4; ++c) {
-                                    const int ncol = tn * kBN + hb * 128 + 32 * c + 8 * o;
-                                    const uint4 sv4 = *reinterpret_cast<const uint4 *>(p.svh + ncol);
-                                    const __half2 *sv = reinterpret_cast<const __half2 *>(&sv4);
-                                    uint32_t pk[4];
-#pragma unroll
-                                    for (int e = 0; e < 8; e += 2) {
-                                        float z[2];
-#pragma unroll
-                                        for (int d = 0; d < 2; ++d) {
-                                            const float a0 = __uint_as_float(u[0 + e + d]);
-                                            const float a1 = __uint_as_float(u[8 + e + d]);
-                                            const float a2 = __uint_as_float(u[16 + e + d]);
-                                            const float a3 = __uint_as_float(u[24 + e + d]);
-                                            const float s01 = a0 + a1, d01 = a0 - a1, s23 = a2 + a3,
-                                                        d23 = a2 - a3;
-                                            // H4 row c: c=0 (+,+,+,+) c=1 (+,-,+,-) c=2 (+,+,-,-) c=3 (+,-,-,+)
-                                            z[d] = c == 0 ? s01 + s23 : c == 1 ? d01 + d23 : c == 2 ? s01 - s23 : d01 - d23;
-                                        }
-                                        const float s = 0.08838834764831845f;
-                                        __half2 h = __floats2half2_rn(z[0] * s * __low2float(sv[e >> 1]),
-                                                                      z[1] * s * __high2float(sv[e >> 1]));
-                                        pk[e >> 1] = *reinterpret_cast<uint32_t *>(&h);
-                                    }
-                                    *reinterpret_cast<uint4 *>(p.y + (int64_t)row * p.n + ncol) =
-                                        make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                                }
-                            }
-                        }
-                    }
-                }
+            if (lane == 0) {
+                mbar_arrive(&bars.bfull[sb]);
+                mbar_arrive(&bars.tempty[st]);
             }
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kWarpMma) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
@@ -493,10 +735,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmParams 
 
 // ------------------------------------------------------------- dispatch ---
 
-static size_t gemm_xt_bytes(int64_t m, int64_t k)
+struct GemmPlan {
+    int64_t tiles, units;
+    int tiles_n, kb_count, ctas;
+    size_t counters, xt, partials, total;  // workspace layout (byte offsets, total size)
+};
+
+static GemmPlan gemm_plan(int64_t m, int64_t k, int64_t n, int sms)
 {
-    const int64_t mp = (m + kBM * kMT - 1) / (kBM * kMT) * (kBM * kMT);
-    return (size_t)mp * (size_t)k * 2;
+    GemmPlan pl;
+    const int64_t tiles_m = (m + kBM * kMT - 1) / (kBM * kMT);
+    pl.tiles_n = (int)(n / kBN);
+    pl.tiles = tiles_m * pl.tiles_n;
+    pl.kb_count = (int)(k / kBK);
+    pl.units = pl.tiles * pl.kb_count;
+    // at least a quarter of a tile's k blocks per CTA: a tile is then split
+    // over at most ~5 CTAs, which bounds the finishing CTA's partial-sum reads
+    const int64_t min_units = pl.kb_count / 4 > 1 ? pl.kb_count / 4 : 1;
+    const int64_t cap = (pl.units + min_units - 1) / min_units;
+    pl.ctas = (int)(cap < sms ? cap : sms);
+    pl.counters = 256;
+    pl.xt = (pl.counters + (size_t)pl.tiles * 4 + 1023) / 1024 * 1024;
+    pl.partials = pl.xt + (size_t)(tiles_m * kBM * kMT) * (size_t)k * 2;
+    pl.total = pl.partials + (size_t)2 * pl.ctas * kPartialFloats * 4;
+    return pl;
 }
 
 template <int K>
@@ -506,8 +768,7 @@ static exl3_status launch_gemm_t(const GemmParams &p, cudaStream_t stream)
     auto kern = gemm_kernel<K>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return EXL3_ERR_CUDA;
-    const int tiles = ((p.m + kBM * kMT - 1) / (kBM * kMT)) * (p.n / kBN);
-    if (launch_kernel(kern, dim3(tiles), dim3(kGemmThreads), (size_t)smem, stream, p) != cudaSuccess)
+    if (launch_kernel(kern, dim3(p.ctas), dim3(kGemmThreads), (size_t)smem, stream, p) != cudaSuccess)
         return EXL3_ERR_CUDA;
     return launch_status();
 }
@@ -518,7 +779,7 @@ extern "C" size_t exl3_gemm_workspace_size(int64_t m, int64_t k, int64_t n, int 
 {
     if (m < 1 || k < 128 || n < 256 || (k % 128) || (n % 256) || K < 1 || K > 8)
         return 0;
-    return 1024 + exl3::gemm_xt_bytes(m, k);
+    return exl3::gemm_plan(m, k, n, exl3::num_sms()).total;
 }
 
 extern "C" exl3_status exl3_gemm(const void *x, const uint16_t *trellis, const void *suh,
@@ -531,12 +792,14 @@ extern "C" exl3_status exl3_gemm(const void *x, const uint16_t *trellis, const v
         return st;
     if (n % kBN)
         return EXL3_ERR_UNSUPPORTED;
-    if (!workspace || !aligned16(workspace) || workspace_bytes < exl3_gemm_workspace_size(m, k, n, K))
+    const GemmPlan pl = gemm_plan(m, k, n, num_sms());
+    if (pl.units * (int64_t)pl.ctas >= ((int64_t)1 << 32))
+        return EXL3_ERR_UNSUPPORTED;  // split the call along m (about 10^14 multiply-adds per call)
+    if (!workspace || !aligned16(workspace) || workspace_bytes < pl.total)
         return EXL3_ERR_WORKSPACE;
     cudaStream_t s = (cudaStream_t)stream;
     unsigned char *ws = (unsigned char *)workspace;
-    unsigned char *xt = ws + 1024;  // 1024-byte aligned relative to a 16-byte aligned base? see below
-    // the tiled x' buffer must be 16-byte aligned for the bulk copies
+    unsigned char *xt = ws + pl.xt;  // 16-byte aligned (1024-byte offset from an aligned base)
     int64_t rot_grid = (m * (k / 128) + 7) / 8;
     if (rot_grid > 148 * 16)
         rot_grid = 148 * 16;
@@ -549,10 +812,16 @@ extern "C" exl3_status exl3_gemm(const void *x, const uint16_t *trellis, const v
     p.trellis = trellis;
     p.svh = (const __half *)svh;
     p.y = (__half *)y;
+    p.partials = reinterpret_cast<float *>(ws + pl.partials);
+    p.counters = reinterpret_cast<uint32_t *>(ws + pl.counters);
+    p.status = (uint32_t *)ws;
     p.m = (int)m;
     p.k = (int)k;
     p.n = (int)n;
-    p.status = (uint32_t *)ws;
+    p.tiles_n = pl.tiles_n;
+    p.kb_count = pl.kb_count;
+    p.units = (uint32_t)pl.units;
+    p.ctas = pl.ctas;
     p.wait_ns = wait_limit_ns();
     p.cb = codebook_constants();
     switch (K) {
