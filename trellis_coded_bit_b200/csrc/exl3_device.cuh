@@ -300,6 +300,24 @@ __device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity, 
     return true;
 }
 
+// Warp-uniform bounded wait for warps that wait often and briefly: every
+// lane polls (one try_wait per poll for the whole warp) and a vote keeps the
+// outcome uniform; the timer is read only every 16 polls.
+__device__ __forceinline__ bool warp_wait_uniform(uint64_t *bar, uint32_t parity, uint64_t limit_ns)
+{
+    if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity)))
+        return true;
+    const uint64_t t0 = global_ns();
+    for (;;) {
+#pragma unroll 1
+        for (int j = 0; j < 16; ++j)
+            if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity)))
+                return true;
+        if (global_ns() - t0 > limit_ns)
+            return false;
+    }
+}
+
 // Warp-uniform bounded wait: lane 0 decides (so a timeout cannot split the
 // warp), then the other lanes observe the completed phase themselves, which
 // cannot move on before this warp releases the stage.

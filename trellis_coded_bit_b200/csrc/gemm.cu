@@ -353,7 +353,8 @@ __device__ __forceinline__ bool gemm_epilogue(const GemmParams &p, GemmBars &bar
     const bool whole = u == tb && se == te;
     const int tm = (int)(t / p.tiles_n), tn = (int)(t - (t / p.tiles_n) * p.tiles_n);
     const int mt_count = (p.m - tm * kBM * kMT) > kBM ? kMT : 1;
-    if (!warp_wait(&bars.acc_full, (uint32_t)seg & 1u, p.wait_ns)) {
+    // a whole k loop can pass before the accumulators are ready: sleep between polls
+    if (!warp_wait(&bars.acc_full, (uint32_t)seg & 1u, p.wait_ns, 1000)) {
         if (lane == 0) {
             record_timeout(p.status);
             *abort_flag = 1;
@@ -704,8 +705,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmParams 
         const int r0 = 2 * (lane & 7);
         for (int i = 0; i < nu; ++i) {
             const int st = i % TS, sb = i % kBStages;
-            if (!warp_wait(&bars.tfull[st], (uint32_t)(i / TS) & 1u, p.wait_ns) ||
-                !warp_wait(&bars.bempty[sb], ((uint32_t)(i / kBStages) & 1u) ^ 1u, p.wait_ns)) {
+            if (!warp_wait_uniform(&bars.tfull[st], (uint32_t)(i / TS) & 1u, p.wait_ns) ||
+                !warp_wait_uniform(&bars.bempty[sb], ((uint32_t)(i / kBStages) & 1u) ^ 1u, p.wait_ns)) {
                 if (lane == 0) {
                     record_timeout(p.status);
                     *abort_flag = 1;
