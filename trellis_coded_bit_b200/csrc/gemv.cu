@@ -50,34 +50,41 @@ constexpr int kGemvThreads = 32 * kGemvWarps;
 // (batches 8mg..8mg+7), quad ba (batches 8mg+ba and 8mg+ba+4) and A-row
 // parity p, a 16-byte record holds the lane's {a0, a1, a2, a3}:
 //   p = 0: {x(8mg+ba), x(8mg+ba+4), 0, 0}     p = 1: {0, 0, x(8mg+ba), x(8mg+ba+4)}
-// with x the rotated activation duplicated in both fp16 halves (absent batches
-// are zero).  Only quads holding a batch < m are stored: rec_slots(m) records
-// per input channel, record (kk, slot) at recs + (kk * slots + slot) * 16.
+// with x the rotated activation duplicated in both fp16 halves (a batch
+// >= m is zero).  Each input channel has rec_slots_for(MG) = 8 MG slots, slot
+// 8mg + 2ba + p, record (kk, slot) at recs + (kk * 8 MG + slot) * 16.  Only
+// quads holding a batch < m are written: a record of an absent quad feeds only
+// A rows of absent batches, whose accumulator rows are never stored, so
+// whatever it holds is harmless.
 __host__ __device__ inline int rec_quads(int m, int mg)
 {
     const int q = m - 8 * mg;
     return q <= 0 ? 0 : (q < 4 ? q : 4);
 }
 
-__host__ __device__ inline int rec_slots(int m)
+__host__ __device__ constexpr int rec_slots_for(int MG)
 {
-    return 2 * (rec_quads(m, 0) + rec_quads(m, 1));
+    return 8 * MG;
+}
+
+__host__ __device__ inline int gemv_mg(int64_t m)
+{
+    return m > 8 ? 2 : 1;
 }
 
 // Workspace layout (bytes): [0, 256) status word; [256, C) arrival counters,
-// one per column block; [C, C+256) a zero record; then the records
-// (k * slots * 16); then the split partials [ncb][max_seg][m][128] f32.
+// one per column block; then the records (k * 8 MG * 16); then the split
+// partials [ncb][max_seg][m][128] f32.
 struct GemvLayout {
-    size_t counters, zero_rec, recs, partials, total;
+    size_t counters, recs, partials, total;
 };
 
 __host__ __device__ inline GemvLayout gemv_layout(int64_t m, int64_t k, int64_t n, int64_t max_seg)
 {
     GemvLayout L;
     L.counters = 256;
-    L.zero_rec = L.counters + (size_t)((n / 128) * 4 + 255) / 256 * 256;
-    L.recs = L.zero_rec + 256;
-    L.partials = L.recs + ((size_t)k * rec_slots((int)m) * 16 + 255) / 256 * 256;
+    L.recs = L.counters + (size_t)((n / 128) * 4 + 255) / 256 * 256;
+    L.partials = L.recs + ((size_t)k * rec_slots_for(gemv_mg(m)) * 16 + 255) / 256 * 256;
     L.total = L.partials + (size_t)(n / 128) * (size_t)max_seg * (size_t)m * 128 * 4;
     return L;
 }
@@ -88,19 +95,16 @@ __host__ __device__ inline GemvLayout gemv_layout(int64_t m, int64_t k, int64_t 
 // batches and writes both parity records of each channel.
 __global__ void __launch_bounds__(256) gemv_rotate_kernel(const __half *__restrict__ x,
                                                           const __half *__restrict__ suh,
-                                                          unsigned char *__restrict__ recs,
-                                                          uint4 *__restrict__ zero_rec, int m, int k)
+                                                          unsigned char *__restrict__ recs, int m, int k)
 {
     grid_dep_wait();    // x may come from the preceding kernel
     grid_dep_launch();  // the main kernel may start streaming weights meanwhile
     const int lane = threadIdx.x & 31;
-    const int slots = rec_slots(m);
+    const int slots = rec_slots_for(gemv_mg(m));
     const int q0 = rec_quads(m, 0), nq = q0 + rec_quads(m, 1);
     const int nblk = k / 128;
     const int64_t jobs = (int64_t)nq * nblk;
     const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    if (blockIdx.x == 0 && threadIdx.x == 0)
-        *zero_rec = make_uint4(0u, 0u, 0u, 0u);
     const float s128 = 0.08838834764831845f;
     for (int64_t job = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); job < jobs; job += warps) {
         const int qd = (int)(job / nblk), blk = (int)(job - (int64_t)qd * nblk);
@@ -126,7 +130,7 @@ __global__ void __launch_bounds__(256) gemv_rotate_kernel(const __half *__restri
             const uint32_t h0 = (uint32_t)__half_as_ushort(__float2half_rn(v0[e] * s128));
             const uint32_t h1 = b1 < m ? (uint32_t)__half_as_ushort(__float2half_rn(v1[e] * s128)) : 0u;
             const uint32_t d0 = h0 | (h0 << 16), d1 = h1 | (h1 << 16);
-            uint4 *rec = reinterpret_cast<uint4 *>(recs + ((int64_t)(c + e) * slots + 2 * qd) * 16);
+            uint4 *rec = reinterpret_cast<uint4 *>(recs + ((int64_t)(c + e) * slots + 8 * mg + 2 * ba) * 16);
             rec[0] = make_uint4(d0, d1, 0u, 0u);  // even A rows
             rec[1] = make_uint4(0u, 0u, d0, d1);  // odd A rows
         }
@@ -140,7 +144,6 @@ struct GemvParams {
     const __half *svh;
     __half *y;
     const unsigned char *recs;
-    const unsigned char *zero_rec;
     float *partials;     // [ncb][max_seg][m][128]
     uint32_t *counters;  // [ncb]
     int m, k, n;
@@ -151,25 +154,24 @@ struct GemvParams {
     Codebook cb;
 };
 
-// Row of tile-row group q for lane t: groups 0,1 take the even rows, groups
-// 2,3 the odd rows, so a group's lanes share the row parity.
-__device__ __forceinline__ int row_of(int q, int t)
-{
-    return 2 * (4 * (q & 1) + t) + (q >> 1);
-}
-
 // Per-warp shared-memory ring: each stage holds one unit -- the 8 tiles of a
 // tile row (each padded to 32K + 16 bytes, which spreads the lanes' row reads
-// over the banks) and that tile row's 16 x slots activation records.
-template <int K>
-struct Stage {
+// over the banks) and that tile row's 16 x 8MG activation records.  The
+// layout is a compile-time function of K and MG, so every shared-memory
+// access of the inner loop is a lane pointer plus an immediate offset.
+template <int K, int MG>
+struct GemvStage {
     static constexpr int kTileStride = 32 * K + 16;
     static constexpr int kTileBytes = 8 * kTileStride;
+    static constexpr int kSlots = rec_slots_for(MG);
+    static constexpr int kRecRowBytes = 16 * kSlots * 16;  // records of one tile row
+    static constexpr int kBytes = (kTileBytes + kRecRowBytes + 127) & ~127;
 };
 
-__host__ __device__ inline int gemv_stage_bytes(int K, int m)
+__host__ __device__ inline int gemv_stage_bytes(int K, int MG)
 {
-    return 8 * (32 * K + 16) + 16 * rec_slots(m) * 16 + 16;  // tiles, records, zero record
+    const int tiles = 8 * (32 * K + 16), recs = 16 * rec_slots_for(MG) * 16;
+    return (tiles + recs + 127) & ~127;
 }
 
 constexpr int kGemvDepth = 3;  // units in flight per warp (one consumed, two loading)
@@ -191,28 +193,42 @@ __device__ __forceinline__ void cp_async_wait()
     asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
-// Per-lane, per-row-group constants: byte offsets (within a stage) of the
-// lane's prefix word, of its row's first 32-bit word, and of its activation
-// record(s) -- the lane's rows never change, so these are computed once.
-struct LaneRows {
-    int pre[4], row[4];
-    int rec[4][2];  // [q][mg] (offset of the record, or of the stage's zero record)
+// Lane (g, t) owns tile g of the unit and, in row group q, the tile row
+// rho(q, t) = 2t + c(q) with c(q) = 8(q & 1) + (q >> 1): groups 0, 1 take
+// the even rows, groups 2, 3 the odd ones, so a group's lanes share the row
+// parity (compile-time bit windows).  Row rho starts at word rho K; its
+// prefix word (rho K - 1) wraps to the tile's last word for rho = 0.
+template <int K>
+__host__ __device__ constexpr int gemv_row_imm(int q)
+{
+    return 4 * (((8 * (q & 1) + (q >> 1)) * K - 1) >> 1);  // floor, -4 for c(q) = 0
+}
+
+// The lane's base pointers into its ring (stage 0): row words, the q = 0
+// prefix word (the wrap lane differs), activation records.
+struct GemvLanePtrs {
+    const unsigned char *row, *pre0, *rec;
 };
 
-// Loads a tile row from shared memory at precomputed offsets, as wide as the
-// row's alignment allows (K = 4: 8 bytes, K = 8: 16 bytes).
-template <int K, int PAR, int N>
-__device__ __forceinline__ void load_row_at(const unsigned char *stage, int pre, int row, uint32_t (&raw)[N])
+// Loads the words of tile row rho(q, t) of stage S: raw[0] the prefix word,
+// then the row's words, as wide as the row's alignment allows.
+template <int K, int MG, int S, int q, int N>
+__device__ __forceinline__ void load_row_q(const GemvLanePtrs &lp, uint32_t (&raw)[N])
 {
+    using St = GemvStage<K, MG>;
+    constexpr int PAR = q >> 1;
     constexpr int P = RowSpan<K, PAR>::P;
     constexpr int N32 = RowSpan<K, PAR>::N32;
-    raw[0] = *reinterpret_cast<const uint32_t *>(stage + pre);
+    constexpr int off = S * St::kBytes + gemv_row_imm<K>(q);
+    const unsigned char *row = lp.row + off;
+    raw[0] = (q == 0) ? *reinterpret_cast<const uint32_t *>(lp.pre0 + S * St::kBytes)
+                      : *reinterpret_cast<const uint32_t *>(row - 4);
     if constexpr (K == 4 && P == 1) {
-        const uint2 v = *reinterpret_cast<const uint2 *>(stage + row);
+        const uint2 v = *reinterpret_cast<const uint2 *>(row);
         raw[1] = v.x;
         raw[2] = v.y;
     } else if constexpr (K == 8 && P == 1) {
-        const uint4 v = *reinterpret_cast<const uint4 *>(stage + row);
+        const uint4 v = *reinterpret_cast<const uint4 *>(row);
         raw[1] = v.x;
         raw[2] = v.y;
         raw[3] = v.z;
@@ -220,44 +236,46 @@ __device__ __forceinline__ void load_row_at(const unsigned char *stage, int pre,
     } else {
 #pragma unroll
         for (int i = 1; i < N32; ++i)
-            raw[i] = *reinterpret_cast<const uint32_t *>(stage + row + 4 * (i - 1));
+            raw[i] = *reinterpret_cast<const uint32_t *>(row + 4 * (i - 1));
     }
 }
 
-template <int K, int MG>
-__device__ __forceinline__ void mac_stage(const unsigned char *stage, const LaneRows &lr, const Codebook &cb,
-                                          float (&acc)[MG][8][4])
+template <int K, int MG, int S, int q>
+__device__ __forceinline__ void mac_row(const GemvLanePtrs &lp, const Codebook &cb, float (&acc)[MG][8][4])
 {
+    using St = GemvStage<K, MG>;
+    constexpr int PAR = q >> 1;
+    constexpr int cq = 8 * (q & 1) + (q >> 1);
+    uint32_t A[MG][4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        uint32_t A[MG][4];
-#pragma unroll
-        for (int mg = 0; mg < MG; ++mg) {
-            const uint4 r = *reinterpret_cast<const uint4 *>(stage + lr.rec[q][mg]);
-            A[mg][0] = r.x;
-            A[mg][1] = r.y;
-            A[mg][2] = r.z;
-            A[mg][3] = r.w;
-        }
-        uint32_t s[16];
-        if (q < 2) {
-            uint32_t raw[RowSpan<K, 0>::N32];
-            load_row_at<K, 0>(stage, lr.pre[q], lr.row[q], raw);
-            row_states<K, RowSpan<K, 0>::P>(raw, s);
-        } else {
-            uint32_t raw[RowSpan<K, 1>::N32];
-            load_row_at<K, 1>(stage, lr.pre[q], lr.row[q], raw);
-            row_states<K, RowSpan<K, 1>::P>(raw, s);
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const uint32_t b0 = codebook_word(s[2 * j], cb);
-            const uint32_t b1 = codebook_word(s[2 * j + 1], cb);
-#pragma unroll
-            for (int mg = 0; mg < MG; ++mg)
-                mma_16816(acc[mg][j], A[mg], b0, b1);
-        }
+    for (int mg = 0; mg < MG; ++mg) {
+        const uint4 r = *reinterpret_cast<const uint4 *>(lp.rec + S * St::kBytes + cq * St::kSlots * 16 + mg * 128);
+        A[mg][0] = r.x;
+        A[mg][1] = r.y;
+        A[mg][2] = r.z;
+        A[mg][3] = r.w;
     }
+    uint32_t raw[RowSpan<K, PAR>::N32];
+    load_row_q<K, MG, S, q>(lp, raw);
+    uint32_t st[16];
+    row_states<K, RowSpan<K, PAR>::P>(raw, st);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const uint32_t b0 = codebook_word(st[2 * j], cb);
+        const uint32_t b1 = codebook_word(st[2 * j + 1], cb);
+#pragma unroll
+        for (int mg = 0; mg < MG; ++mg)
+            mma_16816(acc[mg][j], A[mg], b0, b1);
+    }
+}
+
+template <int K, int MG, int S>
+__device__ __forceinline__ void mac_stage(const GemvLanePtrs &lp, const Codebook &cb, float (&acc)[MG][8][4])
+{
+    mac_row<K, MG, S, 0>(lp, cb, acc);
+    mac_row<K, MG, S, 1>(lp, cb, acc);
+    mac_row<K, MG, S, 2>(lp, cb, acc);
+    mac_row<K, MG, S, 3>(lp, cb, acc);
 }
 
 // CTA owning unit u: the largest c with floor(c U / G) <= u.
@@ -291,102 +309,80 @@ __device__ __forceinline__ void finish_block(const GemvParams &p, const float *r
 template <int K, int MG>
 __global__ void __launch_bounds__(kGemvThreads, MG == 1 ? 2 : 1) gemv_kernel(const GemvParams p)
 {
+    using St = GemvStage<K, MG>;
+    constexpr int SB = St::kBytes;
+    constexpr int kTrChunks = (16 * K + 31) / 32;  // 16-byte trellis chunks per lane per unit
+    constexpr int kRecChunks = St::kRecRowBytes / 16 / 32;
     extern __shared__ __align__(128) unsigned char smem[];
     volatile int *flag = reinterpret_cast<volatile int *>(smem);
     const int m = p.m;
-    const int slots = rec_slots(m);
-    const int stage_bytes = (gemv_stage_bytes(K, m) + 127) & ~127;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    unsigned char *ring = smem + 128 + warp * kGemvDepth * stage_bytes;
-    float *red = reinterpret_cast<float *>(smem + 128 + kGemvWarps * kGemvDepth * stage_bytes);
+    unsigned char *ring = smem + 128 + warp * kGemvDepth * SB;
+    float *red = reinterpret_cast<float *>(smem + 128 + kGemvWarps * kGemvDepth * SB);
 
     const int g = lane >> 2, t = lane & 3;
     const int TR = p.tr_count;
     const int64_t U = p.units;
     const int G = p.ctas;
     const int64_t u0 = (int64_t)blockIdx.x * U / G, u1 = (int64_t)(blockIdx.x + 1) * U / G;
-    // the range as column blocks [cb0, cb1], first block from tile row tb0,
-    // last block up to (excluding) tile row te1
-    const int cb0 = (int)(u0 / TR), tb0 = (int)(u0 - (int64_t)cb0 * TR);
-    const int cb1 = (int)((u1 - 1) / TR), te1 = (int)(u1 - (int64_t)cb1 * TR);
-    auto seg_tb = [&](int c) { return c == cb0 ? tb0 : 0; };
-    auto seg_te = [&](int c) { return c == cb1 ? te1 : TR; };
-    // first unit of this warp at or after column block c (cb > cb1: none)
-    auto first_from = [&](int c, int &tr_out) {
-        for (; c <= cb1; ++c) {
-            const int tr = seg_tb(c) + warp;
-            if (tr < seg_te(c)) {
-                tr_out = tr;
-                return c;
-            }
-        }
-        tr_out = 0;
-        return cb1 + 1;
-    };
-    auto advance = [&](int &c, int &tr) {
-        tr += kGemvWarps;
-        if (tr >= seg_te(c))
-            c = first_from(c + 1, tr);
-    };
+    // the range as column blocks [cb0, cb1]
+    const int cb0 = (int)(u0 / TR), cb1 = (int)((u1 - 1) / TR);
 
+    // lane-constant pointers and copy offsets
+    GemvLanePtrs lp;
+    lp.row = ring + g * St::kTileStride + 4 * (t * K + 1);
+    lp.pre0 = t == 0 ? ring + g * St::kTileStride + 4 * (8 * K - 1)  // row 0: the tile's last word
+                     : lp.row + gemv_row_imm<K>(0) - 4;
+    lp.rec = ring + St::kTileBytes + (2 * t * St::kSlots + g) * 16;
+    unsigned char *tdst[kTrChunks];
+#pragma unroll
+    for (int r = 0; r < kTrChunks; ++r) {
+        const int i = lane + 32 * r;  // chunk i: tile i / 2K, 16-byte piece i % 2K
+        tdst[r] = ring + (i / (2 * K)) * St::kTileStride + (i % (2 * K)) * 16;
+    }
+    const bool last_chunk = (16 * K) % 32 == 0 || lane + 32 * (kTrChunks - 1) < 16 * K;
+
+    // this warp's units: u0 + warp, u0 + warp + 8, ... (< u1), as (column
+    // block, tile row) advanced incrementally; the issue iterator runs
+    // kGemvDepth units ahead of consumption
     const int64_t tile_row_bytes = (int64_t)(p.n >> 4) * 32 * K;  // one tile row of the matrix
-    const int rec_row_bytes = 16 * slots * 16;                   // records of one tile row
-    auto issue = [&](int c, int tr, unsigned char *stage) {
-        if (c <= cb1) {
-            const unsigned char *src =
-                reinterpret_cast<const unsigned char *>(p.trellis) + tr * tile_row_bytes + (int64_t)c * 8 * 32 * K;
-            // 16K chunks of 16 bytes: tile i / 2K, chunk i % 2K
+    const unsigned char *const trellis = reinterpret_cast<const unsigned char *>(p.trellis);
+    int64_t iu = u0 + warp;
+    int icb = (int)(iu / TR), itr = (int)(iu - (int64_t)icb * TR);
+    const unsigned char *isrc = trellis + itr * tile_row_bytes + (int64_t)icb * 8 * 32 * K + lane * 16;
+    const unsigned char *irsrc = p.recs + (int64_t)itr * St::kRecRowBytes + lane * 16;
+    int64_t cu = iu;
+    int ccb = icb;
+
+    auto issue = [&](int stage) {
+        if (iu < u1) {
+            const int so = stage * SB;
 #pragma unroll
-            for (int r = 0; r < (16 * K + 31) / 32; ++r) {
-                const int i = lane + 32 * r;
-                if ((16 * K) % 32 == 0 || i < 16 * K)
-                    cp_async16(stage + (i / (2 * K)) * Stage<K>::kTileStride + (i % (2 * K)) * 16, src + i * 16);
-            }
-            const unsigned char *rsrc = p.recs + (int64_t)tr * rec_row_bytes;
+            for (int r = 0; r < kTrChunks; ++r)
+                if (r < kTrChunks - 1 || last_chunk)
+                    cp_async16(tdst[r] + so, isrc + 512 * r);
 #pragma unroll
-            for (int r = 0; r < 4 * MG; ++r) {  // up to 16 x 8 slots per batch group
-                const int i = lane + 32 * r;
-                if (i < 16 * slots)
-                    cp_async16(stage + Stage<K>::kTileBytes + i * 16, rsrc + i * 16);
+            for (int r = 0; r < kRecChunks; ++r)
+                cp_async16(ring + so + St::kTileBytes + (lane + 32 * r) * 16, irsrc + 512 * r);
+            iu += kGemvWarps;
+            itr += kGemvWarps;
+            isrc += kGemvWarps * tile_row_bytes;
+            irsrc += kGemvWarps * St::kRecRowBytes;
+            if (itr >= TR) {
+                itr -= TR;
+                ++icb;
+                isrc = trellis + itr * tile_row_bytes + (int64_t)icb * 8 * 32 * K + lane * 16;
+                irsrc = p.recs + (int64_t)itr * St::kRecRowBytes + lane * 16;
             }
         }
         cp_async_commit();
     };
 
-    // per-lane offsets within a stage
-    LaneRows lr;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const int rho = row_of(q, t);
-        const int first = (rho * K - 1) >> 1;  // -1 for row 0: the tile's last word (wrap)
-        lr.pre[q] = g * Stage<K>::kTileStride + 4 * (first < 0 ? 8 * K - 1 : first);
-        lr.row[q] = g * Stage<K>::kTileStride + 4 * (first + 1);
-#pragma unroll
-        for (int mg = 0; mg < 2; ++mg) {
-            const int ba = g >> 1;
-            const bool have = mg < MG && ba < rec_quads(m, mg);
-            const int slot = 2 * (mg * rec_quads(m, 0) + ba) + (g & 1);
-            lr.rec[q][mg] = have ? Stage<K>::kTileBytes + (rho * slots + slot) * 16
-                                 : Stage<K>::kTileBytes + rec_row_bytes;  // zero record
-        }
-    }
-
-    // the zero record of every stage of this warp's ring
-    if (lane < kGemvDepth)
-        *reinterpret_cast<uint4 *>(ring + lane * stage_bytes + Stage<K>::kTileBytes + rec_row_bytes) =
-            make_uint4(0u, 0u, 0u, 0u);
-
     // records come from the rotation kernel: wait for it (no-op without PDL)
     grid_dep_wait();
-    int ci, ti;  // issue iterator, kGemvDepth units ahead of consumption
-    ci = first_from(cb0, ti);
-    int cc = ci, tc = ti;  // consume iterator
 #pragma unroll
-    for (int d = 0; d < kGemvDepth; ++d) {
-        issue(ci, ti, ring + d * stage_bytes);
-        if (ci <= cb1)
-            advance(ci, ti);
-    }
+    for (int d = 0; d < kGemvDepth; ++d)
+        issue(d);
     __syncwarp();
 
     const Codebook cb = p.cb;
@@ -401,20 +397,25 @@ __global__ void __launch_bounds__(kGemvThreads, MG == 1 ? 2 : 1) gemv_kernel(con
 
     int st = 0;
     for (int cbk = cb0; cbk <= cb1; ++cbk) {
-        while (cc == cbk) {
+        while (cu < u1 && ccb == cbk) {
             cp_async_wait<kGemvDepth - 1>();
             __syncwarp();
-            unsigned char *stage = ring + st * stage_bytes;
-            mac_stage<K, MG>(stage, lr, cb, acc);
+            if (st == 0)
+                mac_stage<K, MG, 0>(lp, cb, acc);
+            else if (st == 1)
+                mac_stage<K, MG, 1>(lp, cb, acc);
+            else
+                mac_stage<K, MG, 2>(lp, cb, acc);
             __syncwarp();  // every lane is done with the stage before it is refilled
-            issue(ci, ti, stage);
-            if (ci <= cb1)
-                advance(ci, ti);
+            issue(st);
             st = st + 1 == kGemvDepth ? 0 : st + 1;
-            advance(cc, tc);
+            cu += kGemvWarps;
+            // the consumed unit's column block: units advance by 8 < TR tile rows
+            if (cu < u1 && cu >= (int64_t)(ccb + 1) * TR)
+                ++ccb;
         }
-        const int64_t seg_begin = (int64_t)cbk * TR + seg_tb(cbk);
-        const int64_t seg_end = (int64_t)cbk * TR + seg_te(cbk);
+        const int64_t seg_begin = (int64_t)cbk * TR > u0 ? (int64_t)cbk * TR : u0;
+        const int64_t seg_end = (int64_t)(cbk + 1) * TR < u1 ? (int64_t)(cbk + 1) * TR : u1;
 
     // ------------------------------------------- segment end: reduce ---
         // accumulator (mg, j, e): A row i = g (+8 for e >= 2) -> batch 8mg + i/2,
@@ -525,8 +526,7 @@ static GemvPlan gemv_plan(int64_t m, int64_t k, int64_t n, int K, int sms)
     GemvPlan pl;
     const int64_t TR = k / 16, ncb = n / 128;
     pl.units = TR * ncb;
-    pl.smem = 128 + kGemvWarps * kGemvDepth * ((gemv_stage_bytes(K, (int)m) + 127) & ~127) +
-              kGemvWarps * (int)m * 128 * 4;
+    pl.smem = 128 + kGemvWarps * kGemvDepth * gemv_stage_bytes(K, gemv_mg(m)) + kGemvWarps * (int)m * 128 * 4;
     int64_t occ = m <= 8 ? 2 : 1;
     const int64_t occ_smem = (228 * 1024) / (pl.smem + 1024);
     if (occ_smem < occ)
@@ -596,15 +596,14 @@ exl3_status run_gemv(const void *x, const uint16_t *trellis, const void *suh, co
     unsigned char *ws = (unsigned char *)workspace;
 
     // rotation -> records
-    const int64_t jobs = (int64_t)(rec_slots((int)m) / 2) * (k / 128);
+    const int64_t jobs = (int64_t)(rec_quads((int)m, 0) + rec_quads((int)m, 1)) * (k / 128);
     int64_t rgrid = (jobs + 7) / 8;
     if (rgrid > 4 * (int64_t)sms)
         rgrid = 4 * (int64_t)sms;
     if (rgrid < 1)
         rgrid = 1;
     if (launch_kernel(gemv_rotate_kernel, dim3((unsigned)rgrid), dim3(256), 0, stream, (const __half *)x,
-                      (const __half *)suh, ws + L.recs, reinterpret_cast<uint4 *>(ws + L.zero_rec), (int)m,
-                      (int)k) != cudaSuccess ||
+                      (const __half *)suh, ws + L.recs, (int)m, (int)k) != cudaSuccess ||
         launch_status() != EXL3_OK)
         return EXL3_ERR_CUDA;
 
@@ -613,7 +612,6 @@ exl3_status run_gemv(const void *x, const uint16_t *trellis, const void *suh, co
     p.svh = (const __half *)svh;
     p.y = (__half *)y;
     p.recs = ws + L.recs;
-    p.zero_rec = ws + L.zero_rec;
     p.partials = (float *)(ws + L.partials);
     p.counters = (uint32_t *)(ws + L.counters);
     p.m = (int)m;
