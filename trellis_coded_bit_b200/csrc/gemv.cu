@@ -532,9 +532,22 @@ static GemvPlan gemv_plan(int64_t m, int64_t k, int64_t n, int K, int sms)
     if (occ_smem < occ)
         occ = occ_smem > 0 ? occ_smem : 1;
     int64_t G = occ * (int64_t)sms;
-    const int64_t gmax = pl.units / (2 * kGemvWarps);
+    const int64_t gmax = pl.units / (2 * kGemvWarps);  // at least 2 units per warp
     if (G > gmax)
         G = gmax > 0 ? gmax : 1;
+    // A whole number of CTAs per column block aligns the CTA ranges with the
+    // column blocks, so no CTA straddles two (one segment end instead of two,
+    // each about as costly as 8 units).  Take it when the busiest SM's
+    // modelled work (units + 8 per segment end) is lower.
+    const int64_t s_blk = G / ncb;
+    if (s_blk >= 1 && s_blk * ncb != G) {
+        auto cost = [&](int64_t g, int64_t segs) {
+            const int64_t per_sm = (g + sms - 1) / sms;
+            return (pl.units + g - 1) / g * per_sm + 8 * segs * per_sm;
+        };
+        if (cost(s_blk * ncb, 1) < cost(G, 2))
+            G = s_blk * ncb;
+    }
     pl.ctas = (int)G;
     int64_t max_seg = 1;
     for (int64_t cb = 0; cb < ncb; ++cb) {
