@@ -42,6 +42,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-gemm", action="store_true", help="skip the m=2048 GEMM line item")
+    ap.add_argument("--no-stack", action="store_true", help="skip the 70B layer-stack line items")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--profile", default=None,
@@ -349,6 +350,9 @@ def run_ours(args, rank, world, local_rank):
     gemm_info = None
     if not args.no_gemm:
         gemm_info = bench_gemm(exl3, torch, peaks, stream)
+    stack_info = None
+    if not args.no_stack:
+        stack_info = [bench_layer_stack(exl3, torch, peaks, stream, mm) for mm in (1, 32)]
 
     if rank == 0:
         ms = total_ms / args.steps
@@ -393,6 +397,8 @@ def run_ours(args, rank, world, local_rank):
                 "clocks": clocks}
         if gemm_info is not None:
             line["gemm"] = gemm_info
+        if stack_info is not None:
+            line["layer_stack"] = stack_info
         if not args.no_cpu_baseline and world == 1:
             cb = cpu_oracle_sample(layers, args.cpu_seconds)
             cb.pop("seconds", None)
@@ -402,6 +408,55 @@ def run_ours(args, rank, world, local_rank):
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def bench_layer_stack(exl3, torch, peaks, stream, m):
+    """The Llama-3.1-70B decoder-layer linear stack (q, k, v, o at K=4; gate,
+    up, down at K=2; lm_head at K=3) at batch m, one CUDA graph per pass:
+    microseconds per pass and aggregate algorithmic GB/s (weights from HBM:
+    646 MB of trellis, larger than L2)."""
+    specs = [(nm, mm, k, n, K) for (nm, mm, k, n, K, _o) in workloads.LAYER_STACK if mm == m]
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    use_gemv = m <= 16
+    size = exl3.exl3_gemv_workspace_size if use_gemv else exl3.exl3_gemm_workspace_size
+    call = exl3.exl3_gemv if use_gemv else exl3.exl3_gemm
+    ws = exl3.new_workspace(max(size(m, k, n, K) for (_nm, _m, k, n, K) in specs))
+    D = []
+    for i, (nm, mm, k, n, K) in enumerate(specs):
+        L = inputs.make_layer(m, k, n, K, inputs.seed_for(4, i))
+        D.append((dev(L.x), dev(L.trellis), dev(L.suh), dev(L.svh), K,
+                  torch.empty((m, n), dtype=torch.float16, device="cuda")))
+    total_bytes = sum(layer_bytes(m, k, n, K) for (_nm, _m, k, n, K) in specs)
+
+    def one_pass():
+        for x, t, suh, svh, K, y in D:
+            call(x, t, suh, svh, K, y=y, workspace=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            one_pass()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        one_pass()
+    reps = 10
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) / reps * 1e3
+    del g
+    return {"workload": "llama3.1-70b decoder-layer linear stack + lm_head, m=%d (%s)" %
+                        (m, "exl3_gemv" if use_gemv else "exl3_gemm"),
+            "layers": [nm for (nm, _m, _k, _n, _K) in specs], "us_per_pass": us,
+            "algorithmic_bytes_per_pass": total_bytes, "gb_s": total_bytes / (us * 1e-6) / 1e9,
+            "frac_of_hbm_peak": total_bytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"]}
 
 
 def bench_gemm(exl3, torch, peaks, stream):
