@@ -46,8 +46,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--profile", default=None,
-                    help="profiling mode (no timing, no JSON): 'gemv-set' runs the decode GEMV set eagerly "
-                         "warmup+steps times; 'gemm' runs the m=2048 prefill GEMM warmup+steps times; "
+                    help="profiling mode (no timing, no JSON): 'gemv-set' runs the decode GEMV set (one "
+                         "exl3_gemv_multi call, as the bench step) warmup+steps times; 'gemm' runs the m=2048 prefill GEMM warmup+steps times; "
                          "'gemv-layer:k:n:K' runs one m=1 layer")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch without programmatic dependent launch (PDL is valid here: weights are immutable)")
@@ -259,8 +259,16 @@ def run_ours(args, rank, world, local_rank):
                       ws=exl3.new_workspace(ws_bytes), L=L))
     step_bytes = sum(layer_bytes(L.m, L.k, L.n, L.K) for L in layers)
     stream = torch.cuda.Stream()
+    # the step: all 20 layers through one exl3_gemv_multi call (grouped by K
+    # into one rotation + one persistent launch per group)
+    multi = exl3.GemvMulti([(d["x"], d["t"], d["suh"], d["svh"], d["L"].K, d["y"]) for d in D])
+    ws_multi = exl3.new_workspace(multi.workspace_size)
+    n_groups = sum((sum(1 for L in layers if L.K == K) + 15) // 16 for K in set(L.K for L in layers))
 
-    def step(events=None):
+    def step():
+        multi(ws_multi, stream=stream)
+
+    def step_single(events=None):
         for i, d in enumerate(D):
             if events is not None:
                 events[i][0].record(stream)
@@ -273,6 +281,7 @@ def run_ours(args, rank, world, local_rank):
     with torch.cuda.stream(stream):
         for _ in range(2):
             step()
+            step_single()
     stream.synchronize()
 
     # one CUDA graph per step (no nodes but the kernels, so consecutive layers
@@ -286,7 +295,10 @@ def run_ours(args, rank, world, local_rank):
            torch.cuda.Event(enable_timing=True, external=True)) for _ in D]
     graph_ev = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph_ev, stream=stream):
-        step(ev)
+        step_single(ev)
+    graph_single = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_single, stream=stream):
+        step_single()
     for _ in range(args.warmup):
         graph.replay()
     torch.cuda.synchronize()
@@ -312,6 +324,19 @@ def run_ours(args, rank, world, local_rank):
         total_ms = max_over_ranks(total_ms, dist)
         dist.barrier()
 
+    # the same 20 layers as 20 exl3_gemv calls (one graph), for comparison
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            graph_single.replay()
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(args.steps):
+            graph_single.replay()
+        s1.record(stream)
+    torch.cuda.synchronize()
+    single_ms = s0.elapsed_time(s1) / args.steps
+
     # per-kernel durations (L2-cold: the 20-layer rotation exceeds L2)
     kern_samples = []
     for _ in range(5):
@@ -329,8 +354,8 @@ def run_ours(args, rank, world, local_rank):
     def e2e_step():
         for i, d in enumerate(D):
             d["x"].copy_(hx[i], non_blocking=True)
-            exl3.exl3_gemv(d["x"], d["t"], d["suh"], d["svh"], d["L"].K, y=d["y"], workspace=d["ws"],
-                           stream=stream)
+        multi(ws_multi, stream=stream)
+        for i, d in enumerate(D):
             hy[i].copy_(d["y"], non_blocking=True)
 
     with torch.cuda.stream(stream):
@@ -370,14 +395,17 @@ def run_ours(args, rank, world, local_rank):
                 "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
                 "traffic_unit": "bytes per step (ncu dram read + write, all 40 launches of a step)",
                 "algorithmic_bytes_per_step": step_bytes,
-                "kernel": "exl3_gemv = gemv_rotate_kernel + gemv_kernel, 20 layers per step; duration = "
-                          "timed region / steps (one CUDA-graph replay per step)",
+                "kernel": "exl3_gemv_multi over the 20 layers: per K group one gemv_rotate_kernel + one "
+                          "persistent gemv_kernel (%d groups); duration = timed region / steps (one CUDA-graph "
+                          "replay per step)" % n_groups,
                 "peak_source": peaks["source"] + " (burst copy)",
                 "decode_view": {"weights_per_clk_per_sm": w_clk_sm,
                                 "alu_ceiling_weights_per_clk_per_sm": ALU_CEILING_WEIGHTS_PER_CLK_PER_SM,
                                 "frac_of_alu_ceiling": w_clk_sm / ALU_CEILING_WEIGHTS_PER_CLK_PER_SM,
                                 "note": "at m=1 each weight is decoded once; the ALU pipe, not HBM, binds "
                                         "for K <= 6"},
+                "per_layer_calls": {"api": "20 exl3_gemv calls in one graph", "ms_per_step": single_ms,
+                                    "gb_s": job_throughput(step_bytes, world, single_ms)},
                 "per_layer_us_event_bracketed": {"%dx%d_K%d" % (L.k, L.n, L.K): round(t * 1e3, 2)
                                                  for L, t in zip(layers, kernel_ms)}}
         line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -387,9 +415,10 @@ def run_ours(args, rank, world, local_rank):
                            "trellis_bytes_per_step": sum(L.trellis.nbytes for L in layers),
                            "l2": "inputs larger than L2 (398 MB of trellis rotated per step)",
                            "timing": "CUDA graph of one step, CUDA events on the launching stream",
+                           "api": "exl3_gemv_multi (one call for the 20 independent layers)",
                            "launch": "programmatic dependent launch" if not args.no_pdl else "plain",
                            "parallelism": "replica per GPU" if world > 1 else "single GPU"},
-                "roofline": roof, "gpu_launches": 2 * len(D) * args.steps,
+                "roofline": roof, "gpu_launches": 2 * n_groups * args.steps,
                 "e2e": {"value": step_bytes / (e2e_ms * 1e-3) / 1e9 * world, "unit": "GB/s",
                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                         "note": "x copied from pinned host memory and y read back every layer; "
@@ -518,11 +547,11 @@ def run_profile(args):
         else:
             _, k, n, K = what.split(":")
             layers = [inputs.make_layer(1, int(k), int(n), int(K), seed=1)]
-        D = [dict(x=dev(L.x), t=dev(L.trellis), suh=dev(L.suh), svh=dev(L.svh), L=L,
-                  ws=exl3.new_workspace(exl3.exl3_gemv_workspace_size(L.m, L.k, L.n, L.K))) for L in layers]
+        args_l = [(dev(L.x), dev(L.trellis), dev(L.suh), dev(L.svh), L.K, None) for L in layers]
+        multi = exl3.GemvMulti(args_l)
+        ws = exl3.new_workspace(multi.workspace_size)
         for _ in range(args.warmup + args.steps):
-            for d in D:
-                exl3.exl3_gemv(d["x"], d["t"], d["suh"], d["svh"], d["L"].K, workspace=d["ws"])
+            multi(ws)
     torch.cuda.synchronize()
     print("profile run done: %s" % what)
 

@@ -116,6 +116,37 @@ exl3_status exl3_gemv(const void *x, const uint16_t *trellis, const void *suh, c
                       size_t workspace_bytes, void *stream);
 
 /*
+ * exl3_gemv_multi -- several independent layers with the same batch size m
+ * (1 <= m <= 16) in one call: y_i = svh_i .* H(H(x_i .* suh_i) . W_hat_i).
+ * ([GEMM] section 小批量GEMV: the decode-phase GEMV is bandwidth bound, and
+ * a decoder step runs many such layers back to back.)
+ *   layers    HOST array of `count` descriptors (copied during the call; the
+ *             pointers in it are device memory, laid out as for exl3_gemv).
+ *   count     1 .. any; layers are grouped by K and each group (up to 16
+ *             layers) runs as one rotation launch plus one persistent launch
+ *             whose CTAs share out the group's work units evenly, so the
+ *             fixed cost of a launch is paid once per group, not per layer.
+ *   workspace at least exl3_gemv_multi_workspace_size bytes, zero-filled
+ *             once after allocation, not shared by concurrent calls.
+ * Layers must not write one another's inputs (x, trellis, suh, svh).  Results
+ * match exl3_gemv to within the stated tolerance (the split of the sums over
+ * CTAs differs, so the fp32 rounding may too); both are deterministic.
+ * EXL3_ERR_INVALID_ARG if any descriptor is invalid (nothing is launched).
+ */
+typedef struct {
+    const void *x;           /* m x k fp16 */
+    const uint16_t *trellis; /* [k/16][n/16][16K] */
+    const void *suh;         /* k fp16 */
+    const void *svh;         /* n fp16 */
+    void *y;                 /* m x n fp16 (output) */
+    int64_t k, n;
+    int K;
+} exl3_linear;
+size_t exl3_gemv_multi_workspace_size(const exl3_linear *layers, int count, int64_t m);
+exl3_status exl3_gemv_multi(const exl3_linear *layers, int count, int64_t m, void *workspace,
+                            size_t workspace_bytes, void *stream);
+
+/*
  * exl3_gemv_noalloc -- exl3_gemv for callers that cannot allocate device
  * memory.  (The pages have no counterpart: this is a library convenience.)
  *

@@ -106,3 +106,32 @@ def test_hadamard_and_decode_argument_errors():
     assert lib.exl3_decode_tiles(A, B, 24, 16, 4, None) == inv
     assert lib.exl3_decode_tiles(None, B, 16, 16, 4, None) == inv
     assert lib.exl3_workspace_status(None, 0, 0, None) == exl3.EXL3_ERR_WORKSPACE
+
+
+def _multi(descs, m=1, ws=None, wsb=1 << 30):
+    lib = exl3.load()
+    arr = (exl3.Exl3Linear * max(1, len(descs)))(*[exl3.Exl3Linear(*d) for d in descs])
+    return lib.exl3_gemv_multi(arr, len(descs), m, ws, wsb, None)
+
+
+def test_gemv_multi_argument_errors_and_sizes():
+    lib = exl3.load()
+    good = (A, B, C, D, E, 256, 256, 4)
+    inv = exl3.EXL3_ERR_INVALID_ARG
+    assert _multi([]) == inv                                  # no layers
+    assert _multi([good, (A, B, C, D, E, 200, 256, 4)]) == inv  # one bad layer: nothing runs
+    assert _multi([good, (A, B, C, D, MIS, 256, 256, 4)]) == inv
+    assert _multi([good], m=17) == exl3.EXL3_ERR_UNSUPPORTED
+    assert _multi([good], ws=None) == exl3.EXL3_ERR_WORKSPACE
+    assert _multi([good], ws=A, wsb=16) == exl3.EXL3_ERR_WORKSPACE
+
+    def size(descs, m=1):
+        arr = (exl3.Exl3Linear * len(descs))(*[exl3.Exl3Linear(*d) for d in descs])
+        return lib.exl3_gemv_multi_workspace_size(arr, len(descs), m)
+
+    one = size([good])
+    assert 256 <= one <= lib.exl3_gemv_workspace_size(1, 256, 256, 4)
+    # layers of two K values run as two launches, each with its own region
+    two_k = size([good, (A, B, C, D, E, 512, 1024, 2)])
+    assert two_k >= one + size([(A, B, C, D, E, 512, 1024, 2)])
+    assert size([(A, B, C, D, E, 200, 256, 4)]) == 0

@@ -72,50 +72,54 @@ __host__ __device__ inline int gemv_mg(int64_t m)
     return m > 8 ? 2 : 1;
 }
 
-// Workspace layout (bytes): [0, 256) status word; [256, C) arrival counters,
-// one per column block; then the records (k * 8 MG * 16); then the split
-// partials [ncb][max_seg][m][128] f32.
-struct GemvLayout {
-    size_t counters, recs, partials, total;
-};
-
-__host__ __device__ inline GemvLayout gemv_layout(int64_t m, int64_t k, int64_t n, int64_t max_seg)
-{
-    GemvLayout L;
-    L.counters = 256;
-    L.recs = L.counters + (size_t)((n / 128) * 4 + 255) / 256 * 256;
-    L.partials = L.recs + ((size_t)k * rec_slots_for(gemv_mg(m)) * 16 + 255) / 256 * 256;
-    L.total = L.partials + (size_t)(n / 128) * (size_t)max_seg * (size_t)m * 128 * 4;
-    return L;
-}
+// Up to kGemvMaxLayers layers (same K and m) share one launch; their work
+// units and column blocks are numbered consecutively across the layers.
+constexpr int kGemvMaxLayers = 16;
 
 // ------------------------------------------------------ rotation kernel ---
 
-// One warp per (quad, 128-channel block): rotates the quad's one or two
-// batches and writes both parity records of each channel.
-__global__ void __launch_bounds__(256) gemv_rotate_kernel(const __half *__restrict__ x,
-                                                          const __half *__restrict__ suh,
-                                                          unsigned char *__restrict__ recs, int m, int k)
+struct GemvRotLayer {
+    const __half *x;
+    const __half *suh;
+    unsigned char *recs;
+    int k;
+    int64_t job_begin;  // first job of this layer
+};
+
+struct GemvRotParams {
+    GemvRotLayer L[kGemvMaxLayers];
+    int count, m;
+    int64_t jobs;
+};
+
+// One warp per (layer, quad, 128-channel block): rotates the quad's one or
+// two batches and writes both parity records of each channel.
+__global__ void __launch_bounds__(256) gemv_rotate_kernel(const GemvRotParams rp)
 {
     grid_dep_wait();    // x may come from the preceding kernel
     grid_dep_launch();  // the main kernel may start streaming weights meanwhile
     const int lane = threadIdx.x & 31;
+    const int m = rp.m;
     const int slots = rec_slots_for(gemv_mg(m));
-    const int q0 = rec_quads(m, 0), nq = q0 + rec_quads(m, 1);
-    const int nblk = k / 128;
-    const int64_t jobs = (int64_t)nq * nblk;
+    const int q0 = rec_quads(m, 0);
     const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
     const float s128 = 0.08838834764831845f;
-    for (int64_t job = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); job < jobs; job += warps) {
-        const int qd = (int)(job / nblk), blk = (int)(job - (int64_t)qd * nblk);
+    int l = 0;
+    for (int64_t job = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); job < rp.jobs; job += warps) {
+        while (l + 1 < rp.count && job >= rp.L[l + 1].job_begin)
+            ++l;
+        const GemvRotLayer &L = rp.L[l];
+        const int k = L.k, nblk = k / 128;
+        const int64_t lj = job - L.job_begin;
+        const int qd = (int)(lj / nblk), blk = (int)(lj - (int64_t)qd * nblk);
         const int mg = qd >= q0 ? 1 : 0, ba = qd - mg * q0;
         const int b0 = 8 * mg + ba, b1 = b0 + 4;
         const int c = blk * 128 + lane * 4;
-        const uint2 sr = *reinterpret_cast<const uint2 *>(suh + c);
-        const uint2 r0 = *reinterpret_cast<const uint2 *>(x + (int64_t)b0 * k + c);
+        const uint2 sr = *reinterpret_cast<const uint2 *>(L.suh + c);
+        const uint2 r0 = *reinterpret_cast<const uint2 *>(L.x + (int64_t)b0 * k + c);
         uint2 r1 = make_uint2(0u, 0u);
         if (b1 < m)
-            r1 = *reinterpret_cast<const uint2 *>(x + (int64_t)b1 * k + c);
+            r1 = *reinterpret_cast<const uint2 *>(L.x + (int64_t)b1 * k + c);
         const __half2 *sv = reinterpret_cast<const __half2 *>(&sr);
         const __half2 *x0 = reinterpret_cast<const __half2 *>(&r0);
         const __half2 *x1 = reinterpret_cast<const __half2 *>(&r1);
@@ -130,7 +134,7 @@ __global__ void __launch_bounds__(256) gemv_rotate_kernel(const __half *__restri
             const uint32_t h0 = (uint32_t)__half_as_ushort(__float2half_rn(v0[e] * s128));
             const uint32_t h1 = b1 < m ? (uint32_t)__half_as_ushort(__float2half_rn(v1[e] * s128)) : 0u;
             const uint32_t d0 = h0 | (h0 << 16), d1 = h1 | (h1 << 16);
-            uint4 *rec = reinterpret_cast<uint4 *>(recs + ((int64_t)(c + e) * slots + 8 * mg + 2 * ba) * 16);
+            uint4 *rec = reinterpret_cast<uint4 *>(L.recs + ((int64_t)(c + e) * slots + 8 * mg + 2 * ba) * 16);
             rec[0] = make_uint4(d0, d1, 0u, 0u);  // even A rows
             rec[1] = make_uint4(0u, 0u, d0, d1);  // odd A rows
         }
@@ -139,18 +143,24 @@ __global__ void __launch_bounds__(256) gemv_rotate_kernel(const __half *__restri
 
 // ---------------------------------------------------------- main kernel ---
 
-struct GemvParams {
-    const uint16_t *trellis;
+// One layer of a launch.  Global unit u of the layer is unit_begin + cb * TR
+// + tr (column block cb, tile row tr); its column blocks are the launch's
+// column blocks cb_begin .. cb_begin + n/128 - 1.
+struct GemvLayer {
+    const unsigned char *trellis;
     const __half *svh;
     __half *y;
     const unsigned char *recs;
-    float *partials;     // [ncb][max_seg][m][128]
-    uint32_t *counters;  // [ncb]
-    int m, k, n;
-    int tr_count;        // tile rows = k / 16
-    int64_t units;       // (n / 128) * tr_count
-    int ctas;            // grid size G
-    int max_seg;
+    float *partials;     // [n/128][max_seg][m][128]
+    uint32_t *counters;  // [n/128]
+    int64_t unit_begin;
+    int n, tr_count, cb_begin, max_seg;
+};
+
+struct GemvParams {
+    GemvLayer L[kGemvMaxLayers];
+    int count, m, ctas;
+    int64_t units;  // all layers' units
     Codebook cb;
 };
 
@@ -285,16 +295,17 @@ __device__ __forceinline__ int owner_cta(int64_t u, int64_t U, int G)
 }
 
 // Output rotation, svh and fp16 store of one column block's m x 128 y'.
-__device__ __forceinline__ void finish_block(const GemvParams &p, const float *red, int cb, int warp, int lane)
+__device__ __forceinline__ void finish_block(const GemvLayer &L, int m, const float *red, int cb, int warp,
+                                             int lane)
 {
-    for (int b = warp; b < p.m; b += kGemvWarps) {
+    for (int b = warp; b < m; b += kGemvWarps) {
         float v[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e)
             v[e] = red[b * 128 + lane * 4 + e];
         warp_fwht128(v);
         const int c = cb * 128 + lane * 4;
-        const uint2 sr = *reinterpret_cast<const uint2 *>(p.svh + c);
+        const uint2 sr = *reinterpret_cast<const uint2 *>(L.svh + c);
         const __half2 *sv = reinterpret_cast<const __half2 *>(&sr);
         const float s = 0.08838834764831845f;
         __half2 o0 = __floats2half2_rn(v[0] * s * __low2float(sv[0]), v[1] * s * __high2float(sv[0]));
@@ -302,11 +313,24 @@ __device__ __forceinline__ void finish_block(const GemvParams &p, const float *r
         uint2 out;
         out.x = *reinterpret_cast<uint32_t *>(&o0);
         out.y = *reinterpret_cast<uint32_t *>(&o1);
-        *reinterpret_cast<uint2 *>(p.y + (int64_t)b * p.n + c) = out;
+        *reinterpret_cast<uint2 *>(L.y + (int64_t)b * L.n + c) = out;
     }
 }
 
-template <int K, int MG>
+// Position of global unit u: layer l (scanning on from l; always 0 for a
+// single-layer launch), column block cb within it, tile row tr.
+template <bool MULTI>
+__device__ __forceinline__ void gemv_locate(const GemvParams &p, int64_t u, int &l, int &cb, int &tr)
+{
+    while (MULTI && l + 1 < p.count && u >= p.L[l + 1].unit_begin)
+        ++l;
+    const int64_t lu = u - p.L[l].unit_begin;
+    const int TR = p.L[l].tr_count;
+    cb = (int)(lu / TR);
+    tr = (int)(lu - (int64_t)cb * TR);
+}
+
+template <int K, int MG, bool MULTI>
 __global__ void __launch_bounds__(kGemvThreads, MG == 1 ? 2 : 1) gemv_kernel(const GemvParams p)
 {
     using St = GemvStage<K, MG>;
@@ -321,12 +345,9 @@ __global__ void __launch_bounds__(kGemvThreads, MG == 1 ? 2 : 1) gemv_kernel(con
     float *red = reinterpret_cast<float *>(smem + 128 + kGemvWarps * kGemvDepth * SB);
 
     const int g = lane >> 2, t = lane & 3;
-    const int TR = p.tr_count;
     const int64_t U = p.units;
     const int G = p.ctas;
     const int64_t u0 = (int64_t)blockIdx.x * U / G, u1 = (int64_t)(blockIdx.x + 1) * U / G;
-    // the range as column blocks [cb0, cb1]
-    const int cb0 = (int)(u0 / TR), cb1 = (int)((u1 - 1) / TR);
 
     // lane-constant pointers and copy offsets
     GemvLanePtrs lp;
@@ -342,17 +363,28 @@ __global__ void __launch_bounds__(kGemvThreads, MG == 1 ? 2 : 1) gemv_kernel(con
     }
     const bool last_chunk = (16 * K) % 32 == 0 || lane + 32 * (kTrChunks - 1) < 16 * K;
 
-    // this warp's units: u0 + warp, u0 + warp + 8, ... (< u1), as (column
-    // block, tile row) advanced incrementally; the issue iterator runs
+    // this warp's units: u0 + warp, u0 + warp + 8, ... (< u1), as (layer,
+    // column block, tile row) advanced incrementally; the issue iterator runs
     // kGemvDepth units ahead of consumption
-    const int64_t tile_row_bytes = (int64_t)(p.n >> 4) * 32 * K;  // one tile row of the matrix
-    const unsigned char *const trellis = reinterpret_cast<const unsigned char *>(p.trellis);
     int64_t iu = u0 + warp;
-    int icb = (int)(iu / TR), itr = (int)(iu - (int64_t)icb * TR);
-    const unsigned char *isrc = trellis + itr * tile_row_bytes + (int64_t)icb * 8 * 32 * K + lane * 16;
-    const unsigned char *irsrc = p.recs + (int64_t)itr * St::kRecRowBytes + lane * 16;
+    int il = 0, icb = 0, itr = 0;
+    gemv_locate<MULTI>(p, iu < u1 ? iu : u0, il, icb, itr);
+    int64_t tile_row_bytes = 0;
+    int itr_lim = 0, incb = 0;  // the issue layer's tile rows and column blocks
+    const unsigned char *isrc = nullptr, *irsrc = nullptr;
+    auto point = [&]() {
+        const GemvLayer &L = p.L[il];
+        itr_lim = L.tr_count;
+        incb = L.n >> 7;
+        tile_row_bytes = (int64_t)(L.n >> 4) * 32 * K;  // one tile row of the layer's matrix
+        isrc = L.trellis + itr * tile_row_bytes + (int64_t)icb * 8 * 32 * K + lane * 16;
+        irsrc = L.recs + (int64_t)itr * St::kRecRowBytes + lane * 16;
+    };
+    point();
     int64_t cu = iu;
-    int ccb = icb;
+    int cl = il, ccb = icb, ctr = itr;  // consumed unit: layer, column block, tile row
+    int cg = p.L[il].cb_begin + icb;    // consumed unit's global column block
+    int ctr_lim = itr_lim, cncb = incb;  // the consumed unit's layer: tile rows, column blocks
 
     auto issue = [&](int stage) {
         if (iu < u1) {
@@ -368,11 +400,15 @@ __global__ void __launch_bounds__(kGemvThreads, MG == 1 ? 2 : 1) gemv_kernel(con
             itr += kGemvWarps;
             isrc += kGemvWarps * tile_row_bytes;
             irsrc += kGemvWarps * St::kRecRowBytes;
-            if (itr >= TR) {
-                itr -= TR;
-                ++icb;
-                isrc = trellis + itr * tile_row_bytes + (int64_t)icb * 8 * 32 * K + lane * 16;
-                irsrc = p.recs + (int64_t)itr * St::kRecRowBytes + lane * 16;
+            if (itr >= itr_lim) {  // next column block, perhaps of the next layer (units advance by 8 <= TR)
+                itr -= itr_lim;
+                if (++icb == incb) {
+                    icb = 0;
+                    if (MULTI)
+                        ++il;
+                }
+                if (iu < u1)
+                    point();
             }
         }
         cp_async_commit();
@@ -395,9 +431,21 @@ __global__ void __launch_bounds__(kGemvThreads, MG == 1 ? 2 : 1) gemv_kernel(con
             for (int e = 0; e < 4; ++e)
                 acc[a][j][e] = 0.f;
 
+    // the CTA's range as global column blocks [g0, g1]
+    int l0 = 0, c0 = 0, r0 = 0, l1 = 0, c1 = 0, r1 = 0;
+    gemv_locate<MULTI>(p, u0, l0, c0, r0);
+    l1 = l0;
+    gemv_locate<MULTI>(p, u1 - 1, l1, c1, r1);
+    const int g0 = p.L[l0].cb_begin + c0, g1 = p.L[l1].cb_begin + c1;
+    int sl = l0;  // layer of the current segment's column block
     int st = 0;
-    for (int cbk = cb0; cbk <= cb1; ++cbk) {
-        while (cu < u1 && ccb == cbk) {
+    for (int gk = g0; gk <= g1; ++gk) {
+        while (MULTI && sl + 1 < p.count && gk >= p.L[sl + 1].cb_begin)
+            ++sl;
+        const GemvLayer &SL = p.L[sl];
+        const int TR = SL.tr_count;
+        const int cbk = gk - SL.cb_begin;  // column block within the layer
+        while (cu < u1 && cg == gk) {
             cp_async_wait<kGemvDepth - 1>();
             __syncwarp();
             if (st == 0)
@@ -410,12 +458,25 @@ __global__ void __launch_bounds__(kGemvThreads, MG == 1 ? 2 : 1) gemv_kernel(con
             issue(st);
             st = st + 1 == kGemvDepth ? 0 : st + 1;
             cu += kGemvWarps;
-            // the consumed unit's column block: units advance by 8 < TR tile rows
-            if (cu < u1 && cu >= (int64_t)(ccb + 1) * TR)
-                ++ccb;
+            // the consumed unit's column block: units advance by 8 <= TR tile rows
+            ctr += kGemvWarps;
+            if (ctr >= ctr_lim) {
+                ctr -= ctr_lim;
+                if (++ccb == cncb) {
+                    ccb = 0;
+                    if (MULTI)
+                        ++cl;
+                    if (MULTI && cu < u1) {
+                        ctr_lim = p.L[cl].tr_count;
+                        cncb = p.L[cl].n >> 7;
+                    }
+                }
+                cg = cu < u1 ? p.L[cl].cb_begin + ccb : cg + 1;
+            }
         }
-        const int64_t seg_begin = (int64_t)cbk * TR > u0 ? (int64_t)cbk * TR : u0;
-        const int64_t seg_end = (int64_t)(cbk + 1) * TR < u1 ? (int64_t)(cbk + 1) * TR : u1;
+        const int64_t blk_begin = SL.unit_begin + (int64_t)cbk * TR, blk_end = blk_begin + TR;
+        const int64_t seg_begin = blk_begin > u0 ? blk_begin : u0;
+        const int64_t seg_end = blk_end < u1 ? blk_end : u1;
 
     // ------------------------------------------- segment end: reduce ---
         // accumulator (mg, j, e): A row i = g (+8 for e >= 2) -> batch 8mg + i/2,
@@ -444,21 +505,21 @@ __global__ void __launch_bounds__(kGemvThreads, MG == 1 ? 2 : 1) gemv_kernel(con
             red[e] = sum;
         }
         __syncthreads();
-        const bool whole = seg_begin == (int64_t)cbk * TR && seg_end == ((int64_t)cbk + 1) * TR;
+        const bool whole = seg_begin == blk_begin && seg_end == blk_end;
         if (whole) {
-            finish_block(p, red, cbk, warp, lane);
+            finish_block(SL, m, red, cbk, warp, lane);
         } else {
-            const int c_first = owner_cta((int64_t)cbk * TR, U, G);
-            const int c_last = owner_cta(((int64_t)cbk + 1) * TR - 1, U, G);
+            const int c_first = owner_cta(blk_begin, U, G);
+            const int c_last = owner_cta(blk_end - 1, U, G);
             const int nseg = c_last - c_first + 1;
             const int j = (int)blockIdx.x - c_first;
-            float *part = p.partials + ((int64_t)cbk * p.max_seg) * m * 128;
+            float *part = SL.partials + ((int64_t)cbk * SL.max_seg) * m * 128;
             for (int e = tid; e < m * 128; e += kGemvThreads)
                 part[(int64_t)j * m * 128 + e] = red[e];
             __threadfence();
             __syncthreads();
             if (tid == 0) {
-                const uint32_t ticket = atomicAdd(&p.counters[cbk], 1u);
+                const uint32_t ticket = atomicAdd(&SL.counters[cbk], 1u);
                 *flag = (ticket == (uint32_t)(nseg - 1)) ? 1 : 0;
             }
             __syncthreads();
@@ -478,9 +539,9 @@ __global__ void __launch_bounds__(kGemvThreads, MG == 1 ? 2 : 1) gemv_kernel(con
                     red[e] = (((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]))) + tail;
                 }
                 if (tid == 0)
-                    p.counters[cbk] = 0u;
+                    SL.counters[cbk] = 0u;
                 __syncthreads();
-                finish_block(p, red, cbk, warp, lane);
+                finish_block(SL, m, red, cbk, warp, lane);
             }
         }
         __syncthreads();  // red is reused by the next segment
@@ -489,11 +550,6 @@ __global__ void __launch_bounds__(kGemvThreads, MG == 1 ? 2 : 1) gemv_kernel(con
 }
 
 // ------------------------------------------------------------- dispatch ---
-
-struct GemvPlan {
-    int ctas, max_seg, smem;
-    int64_t units;
-};
 
 static int g_num_sms = 0;
 
@@ -517,15 +573,33 @@ static int64_t owner_cta_host(int64_t u, int64_t U, int64_t G)
     return ((u + 1) * G - 1) / U;
 }
 
+// Plan of one launch over `count` layers (same K, same m): grid, shared
+// memory, and the workspace layout -- [0, 256) status word; the layers'
+// arrival counters (one per column block, consecutive); then per layer its
+// activation records (k * 8 MG * 16) and split partials [n/128][max_seg][m][128].
+struct GemvGroupPlan {
+    int ctas, smem;
+    int64_t units;
+    int64_t unit_begin[kGemvMaxLayers];
+    int cb_begin[kGemvMaxLayers], max_seg[kGemvMaxLayers];
+    size_t counters[kGemvMaxLayers], recs[kGemvMaxLayers], partials[kGemvMaxLayers], total;
+};
+
 // Grid: every CTA resident at once -- resident CTAs per SM from the register
 // budget (2 for m <= 8, 1 above) and the shared memory (228 KB per SM, 1 KB
 // reserved per CTA) -- but at least two units per warp; max_seg = the most
-// CTAs any column block is split over.
-static GemvPlan gemv_plan(int64_t m, int64_t k, int64_t n, int K, int sms)
+// CTAs any column block of the layer is split over.
+static GemvGroupPlan gemv_group_plan(const int64_t *k, const int64_t *n, int count, int64_t m, int K, int sms)
 {
-    GemvPlan pl;
-    const int64_t TR = k / 16, ncb = n / 128;
-    pl.units = TR * ncb;
+    GemvGroupPlan pl;
+    pl.units = 0;
+    int cb = 0;
+    for (int l = 0; l < count; ++l) {
+        pl.unit_begin[l] = pl.units;
+        pl.cb_begin[l] = cb;
+        pl.units += (k[l] / 16) * (n[l] / 128);
+        cb += (int)(n[l] / 128);
+    }
     pl.smem = 128 + kGemvWarps * kGemvDepth * gemv_stage_bytes(K, gemv_mg(m)) + kGemvWarps * (int)m * 128 * 4;
     int64_t occ = m <= 8 ? 2 : 1;
     const int64_t occ_smem = (228 * 1024) / (pl.smem + 1024);
@@ -535,27 +609,46 @@ static GemvPlan gemv_plan(int64_t m, int64_t k, int64_t n, int K, int sms)
     const int64_t gmax = pl.units / (2 * kGemvWarps);  // at least 2 units per warp
     if (G > gmax)
         G = gmax > 0 ? gmax : 1;
-    // A whole number of CTAs per column block aligns the CTA ranges with the
-    // column blocks, so no CTA straddles two (one segment end instead of two,
-    // each about as costly as 8 units).  Take it when the busiest SM's
-    // modelled work (units + 8 per segment end) is lower.
-    const int64_t s_blk = G / ncb;
-    if (s_blk >= 1 && s_blk * ncb != G) {
-        auto cost = [&](int64_t g, int64_t segs) {
-            const int64_t per_sm = (g + sms - 1) / sms;
-            return (pl.units + g - 1) / g * per_sm + 8 * segs * per_sm;
-        };
-        if (cost(s_blk * ncb, 1) < cost(G, 2))
-            G = s_blk * ncb;
+    if (count == 1) {
+        // A whole number of CTAs per column block aligns the CTA ranges with
+        // the column blocks, so no CTA straddles two (one segment end instead
+        // of two, each about as costly as 8 units).  Take it when the busiest
+        // SM's modelled work (units + 8 per segment end) is lower.
+        const int64_t ncb = n[0] / 128;
+        const int64_t s_blk = G / ncb;
+        if (s_blk >= 1 && s_blk * ncb != G) {
+            auto cost = [&](int64_t g, int64_t segs) {
+                const int64_t per_sm = (g + sms - 1) / sms;
+                return (pl.units + g - 1) / g * per_sm + 8 * segs * per_sm;
+            };
+            if (cost(s_blk * ncb, 1) < cost(G, 2))
+                G = s_blk * ncb;
+        }
     }
     pl.ctas = (int)G;
-    int64_t max_seg = 1;
-    for (int64_t cb = 0; cb < ncb; ++cb) {
-        const int64_t s = owner_cta_host((cb + 1) * TR - 1, pl.units, G) - owner_cta_host(cb * TR, pl.units, G) + 1;
-        if (s > max_seg)
-            max_seg = s;
+    size_t off = 256;
+    for (int l = 0; l < count; ++l) {
+        pl.counters[l] = off;
+        off += (size_t)(n[l] / 128) * 4;
     }
-    pl.max_seg = (int)max_seg;
+    off = (off + 255) / 256 * 256;
+    for (int l = 0; l < count; ++l) {
+        const int64_t TR = k[l] / 16, ncb = n[l] / 128;
+        int64_t max_seg = 1;
+        for (int64_t c = 0; c < ncb; ++c) {
+            const int64_t b0 = pl.unit_begin[l] + c * TR;
+            const int64_t s = owner_cta_host(b0 + TR - 1, pl.units, G) - owner_cta_host(b0, pl.units, G) + 1;
+            max_seg = s > max_seg ? s : max_seg;
+        }
+        pl.max_seg[l] = (int)max_seg;
+        pl.recs[l] = off;
+        off += ((size_t)k[l] * rec_slots_for(gemv_mg(m)) * 16 + 255) / 256 * 256;
+    }
+    for (int l = 0; l < count; ++l) {
+        pl.partials[l] = off;
+        off += ((size_t)(n[l] / 128) * (size_t)pl.max_seg[l] * (size_t)m * 128 * 4 + 255) / 256 * 256;
+    }
+    pl.total = off;
     return pl;
 }
 
@@ -563,8 +656,7 @@ size_t gemv_workspace_bytes(int64_t m, int64_t k, int64_t n, int sms)
 {
     size_t most = 0;
     for (int K = 1; K <= 8; ++K) {
-        const GemvPlan pl = gemv_plan(m, k, n, K, sms);
-        const size_t b = gemv_layout(m, k, n, pl.max_seg).total;
+        const size_t b = gemv_group_plan(&k, &n, 1, m, K, sms).total;
         most = b > most ? b : most;
     }
     return most;
@@ -573,7 +665,7 @@ size_t gemv_workspace_bytes(int64_t m, int64_t k, int64_t n, int sms)
 template <int K, int MG>
 static exl3_status launch_gemv_t(const GemvParams &p, int smem, cudaStream_t stream)
 {
-    auto kern = gemv_kernel<K, MG>;
+    auto kern = p.count > 1 ? gemv_kernel<K, MG, true> : gemv_kernel<K, MG, false>;
     if (smem > 48 * 1024 &&
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return EXL3_ERR_CUDA;
@@ -597,47 +689,117 @@ static exl3_status launch_gemv_k(const GemvParams &p, int K, int smem, cudaStrea
     }
 }
 
-exl3_status run_gemv(const void *x, const uint16_t *trellis, const void *suh, const void *svh,
-                     void *y, int64_t m, int64_t k, int64_t n, int K, void *workspace,
-                     size_t workspace_bytes, cudaStream_t stream)
+// One launch pair (rotation, main kernel) over up to kGemvMaxLayers layers of
+// the same K, with the workspace region `ws` laid out by gemv_group_plan.
+static exl3_status run_gemv_group(const exl3_linear *const *layers, int count, int64_t m, int K,
+                                  unsigned char *ws, size_t ws_bytes, cudaStream_t stream)
 {
     const int sms = num_sms();
-    const GemvPlan pl = gemv_plan(m, k, n, K, sms);
-    const GemvLayout L = gemv_layout(m, k, n, pl.max_seg);
-    if (!workspace || !aligned16(workspace) || workspace_bytes < L.total)
+    int64_t k[kGemvMaxLayers], n[kGemvMaxLayers];
+    for (int l = 0; l < count; ++l) {
+        k[l] = layers[l]->k;
+        n[l] = layers[l]->n;
+    }
+    const GemvGroupPlan pl = gemv_group_plan(k, n, count, m, K, sms);
+    if (!ws || !aligned16(ws) || ws_bytes < pl.total)
         return EXL3_ERR_WORKSPACE;
-    unsigned char *ws = (unsigned char *)workspace;
 
     // rotation -> records
-    const int64_t jobs = (int64_t)(rec_quads((int)m, 0) + rec_quads((int)m, 1)) * (k / 128);
+    GemvRotParams rp;
+    rp.count = count;
+    rp.m = (int)m;
+    int64_t jobs = 0;
+    const int quads = rec_quads((int)m, 0) + rec_quads((int)m, 1);
+    for (int l = 0; l < count; ++l) {
+        rp.L[l].x = (const __half *)layers[l]->x;
+        rp.L[l].suh = (const __half *)layers[l]->suh;
+        rp.L[l].recs = ws + pl.recs[l];
+        rp.L[l].k = (int)k[l];
+        rp.L[l].job_begin = jobs;
+        jobs += (int64_t)quads * (k[l] / 128);
+    }
+    rp.jobs = jobs;
     int64_t rgrid = (jobs + 7) / 8;
     if (rgrid > 4 * (int64_t)sms)
         rgrid = 4 * (int64_t)sms;
     if (rgrid < 1)
         rgrid = 1;
-    if (launch_kernel(gemv_rotate_kernel, dim3((unsigned)rgrid), dim3(256), 0, stream, (const __half *)x,
-                      (const __half *)suh, ws + L.recs, (int)m, (int)k) != cudaSuccess ||
+    if (launch_kernel(gemv_rotate_kernel, dim3((unsigned)rgrid), dim3(256), 0, stream, rp) != cudaSuccess ||
         launch_status() != EXL3_OK)
         return EXL3_ERR_CUDA;
 
     GemvParams p;
-    p.trellis = trellis;
-    p.svh = (const __half *)svh;
-    p.y = (__half *)y;
-    p.recs = ws + L.recs;
-    p.partials = (float *)(ws + L.partials);
-    p.counters = (uint32_t *)(ws + L.counters);
+    p.count = count;
     p.m = (int)m;
-    p.k = (int)k;
-    p.n = (int)n;
-    p.tr_count = (int)(k / 16);
-    p.units = pl.units;
     p.ctas = pl.ctas;
-    p.max_seg = pl.max_seg;
+    p.units = pl.units;
     p.cb = codebook_constants();
+    for (int l = 0; l < count; ++l) {
+        GemvLayer &L = p.L[l];
+        L.trellis = reinterpret_cast<const unsigned char *>(layers[l]->trellis);
+        L.svh = (const __half *)layers[l]->svh;
+        L.y = (__half *)layers[l]->y;
+        L.recs = ws + pl.recs[l];
+        L.partials = reinterpret_cast<float *>(ws + pl.partials[l]);
+        L.counters = reinterpret_cast<uint32_t *>(ws + pl.counters[l]);
+        L.unit_begin = pl.unit_begin[l];
+        L.n = (int)n[l];
+        L.tr_count = (int)(k[l] / 16);
+        L.cb_begin = pl.cb_begin[l];
+        L.max_seg = pl.max_seg[l];
+    }
     if (m <= 8)
         return launch_gemv_k<1>(p, K, pl.smem, stream);
     return launch_gemv_k<2>(p, K, pl.smem, stream);
+}
+
+exl3_status run_gemv(const void *x, const uint16_t *trellis, const void *suh, const void *svh,
+                     void *y, int64_t m, int64_t k, int64_t n, int K, void *workspace,
+                     size_t workspace_bytes, cudaStream_t stream)
+{
+    exl3_linear d;
+    d.x = x;
+    d.trellis = trellis;
+    d.suh = suh;
+    d.svh = svh;
+    d.y = y;
+    d.k = k;
+    d.n = n;
+    d.K = K;
+    const exl3_linear *one = &d;
+    return run_gemv_group(&one, 1, m, K, (unsigned char *)workspace, workspace_bytes, stream);
+}
+
+// The layers of a multi call, grouped by K (in call order) into launches of
+// at most kGemvMaxLayers; calls f(group, count, K, workspace offset, bytes).
+template <typename F>
+static exl3_status for_each_gemv_group(const exl3_linear *layers, int count, int64_t m, F &&f)
+{
+    const int sms = num_sms();
+    size_t off = 0;
+    for (int K = 1; K <= 8; ++K) {
+        const exl3_linear *grp[kGemvMaxLayers];
+        int cnt = 0;
+        for (int i = 0; i <= count; ++i) {
+            const bool flush = (i == count && cnt > 0) || cnt == kGemvMaxLayers;
+            if (flush) {
+                int64_t k[kGemvMaxLayers], n[kGemvMaxLayers];
+                for (int l = 0; l < cnt; ++l) {
+                    k[l] = grp[l]->k;
+                    n[l] = grp[l]->n;
+                }
+                const size_t bytes = gemv_group_plan(k, n, cnt, m, K, sms).total;
+                const exl3_status st = f(grp, cnt, K, off, bytes);
+                if (st != EXL3_OK)
+                    return st;
+                off += (bytes + 255) / 256 * 256;
+                cnt = 0;
+            }
+            if (i < count && layers[i].K == K)
+                grp[cnt++] = &layers[i];
+        }
+    }
+    return EXL3_OK;
 }
 
 }  // namespace exl3
@@ -661,6 +823,49 @@ extern "C" exl3_status exl3_gemv(const void *x, const uint16_t *trellis, const v
         return EXL3_ERR_UNSUPPORTED;
     return run_gemv(x, trellis, suh, svh, y, m, k, n, K, workspace, workspace_bytes,
                     (cudaStream_t)stream);
+}
+
+static exl3_status check_multi(const exl3_linear *layers, int count, int64_t m)
+{
+    using namespace exl3;
+    if (!layers || count < 1)
+        return EXL3_ERR_INVALID_ARG;
+    for (int i = 0; i < count; ++i) {
+        const exl3_linear &d = layers[i];
+        const exl3_status st = check_linear_args(d.x, d.trellis, d.suh, d.svh, d.y, m, d.k, d.n, d.K);
+        if (st != EXL3_OK)
+            return st;
+    }
+    return m > 16 ? EXL3_ERR_UNSUPPORTED : EXL3_OK;
+}
+
+extern "C" size_t exl3_gemv_multi_workspace_size(const exl3_linear *layers, int count, int64_t m)
+{
+    using namespace exl3;
+    if (check_multi(layers, count, m) != EXL3_OK)
+        return 0;
+    size_t total = 0;
+    for_each_gemv_group(layers, count, m, [&](const exl3_linear *const *, int, int, size_t off, size_t bytes) {
+        total = off + (bytes + 255) / 256 * 256;
+        return EXL3_OK;
+    });
+    return total;
+}
+
+extern "C" exl3_status exl3_gemv_multi(const exl3_linear *layers, int count, int64_t m, void *workspace,
+                                       size_t workspace_bytes, void *stream)
+{
+    using namespace exl3;
+    const exl3_status st = check_multi(layers, count, m);
+    if (st != EXL3_OK)
+        return st;
+    if (!workspace || !aligned16(workspace) || workspace_bytes < exl3_gemv_multi_workspace_size(layers, count, m))
+        return EXL3_ERR_WORKSPACE;
+    unsigned char *ws = (unsigned char *)workspace;
+    return for_each_gemv_group(layers, count, m,
+                               [&](const exl3_linear *const *grp, int cnt, int K, size_t off, size_t bytes) {
+                                   return run_gemv_group(grp, cnt, m, K, ws + off, bytes, (cudaStream_t)stream);
+                               });
 }
 
 // ------------------------------------------------ no-allocation variant ---

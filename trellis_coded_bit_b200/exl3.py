@@ -22,7 +22,8 @@ EXL3_ERR_TIMEOUT = 5
 
 # Every symbol the public headers declare.
 EXPORTED = ["exl3_status_string", "exl3_version", "exl3_hadamard", "exl3_decode_tiles",
-            "exl3_gemv_workspace_size", "exl3_gemv", "exl3_gemv_noalloc_max_scratch",
+            "exl3_gemv_workspace_size", "exl3_gemv", "exl3_gemv_multi_workspace_size", "exl3_gemv_multi",
+            "exl3_gemv_noalloc_max_scratch",
             "exl3_gemv_noalloc", "exl3_gemm_workspace_size", "exl3_gemm",
             "exl3_workspace_status", "exl3_set_launch_flags", "exl3_launch_flags",
             "exl3_debug_set_wait_limit_ns", "exl3_debug_wait_limit_ns"]
@@ -31,6 +32,13 @@ EXL3_LAUNCH_PDL = 1
 
 _lib = None
 _lock = threading.Lock()
+
+
+class Exl3Linear(ctypes.Structure):
+    """The C struct exl3_linear: one layer of an exl3_gemv_multi call."""
+    _fields_ = [("x", ctypes.c_void_p), ("trellis", ctypes.c_void_p), ("suh", ctypes.c_void_p),
+                ("svh", ctypes.c_void_p), ("y", ctypes.c_void_p), ("k", ctypes.c_int64),
+                ("n", ctypes.c_int64), ("K", ctypes.c_int)]
 
 
 class Exl3Error(RuntimeError):
@@ -69,6 +77,10 @@ def load(build_if_needed=True):
         for name in ("exl3_gemv", "exl3_gemm"):
             getattr(lib, name).argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, ci, vp, sz, vp]
             getattr(lib, name).restype = ci
+        lib.exl3_gemv_multi_workspace_size.argtypes = [ctypes.POINTER(Exl3Linear), ci, i64]
+        lib.exl3_gemv_multi_workspace_size.restype = sz
+        lib.exl3_gemv_multi.argtypes = [ctypes.POINTER(Exl3Linear), ci, i64, vp, sz, vp]
+        lib.exl3_gemv_multi.restype = ci
         lib.exl3_gemv_noalloc_max_scratch.argtypes = []
         lib.exl3_gemv_noalloc_max_scratch.restype = sz
         lib.exl3_gemv_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, ci, vp]
@@ -173,6 +185,58 @@ def _linear(fn, name, x, trellis, suh, svh, K, y, workspace, stream):
 def exl3_gemv(x, trellis, suh, svh, K, y=None, workspace=None, stream=None):
     """y = svh .* H(H(x .* suh) W_hat) for 1 <= m <= 16 (memory-bound path)."""
     return _linear(load().exl3_gemv, "exl3_gemv", x, trellis, suh, svh, K, y, workspace, stream)
+
+
+def _linear_array(layers, m):
+    """layers: sequence of (x, trellis, suh, svh, K, y) CUDA tensors (y may be None)."""
+    arr = (Exl3Linear * len(layers))()
+    ys = []
+    for i, (x, trellis, suh, svh, K, y) in enumerate(layers):
+        if x.shape[0] != m:
+            raise ValueError("every layer of a multi call has the same batch size m")
+        k, n = x.shape[1], svh.numel()
+        if y is None:
+            y = torch.empty((m, n), dtype=torch.float16, device=x.device)
+        arr[i] = Exl3Linear(_dev(x, torch.float16, "x"), _dev(trellis, torch.uint16, "trellis"),
+                            _dev(suh, torch.float16, "suh"), _dev(svh, torch.float16, "svh"),
+                            _dev(y, torch.float16, "y"), k, n, int(K))
+        ys.append(y)
+    return arr, ys
+
+
+def exl3_gemv_multi_workspace_size(layers, m):
+    """Workspace bytes for exl3_gemv_multi over `layers` (see exl3_gemv_multi)."""
+    arr, _ = _linear_array(layers, m)
+    return int(load().exl3_gemv_multi_workspace_size(arr, len(layers), m))
+
+
+def exl3_gemv_multi(layers, workspace=None, stream=None):
+    """Several independent layers (same m <= 16) in one call: each entry is
+    (x, trellis, suh, svh, K, y-or-None); returns the list of y."""
+    m = layers[0][0].shape[0]
+    arr, ys = _linear_array(layers, m)
+    if workspace is None:
+        raise ValueError("exl3_gemv_multi needs a workspace (exl3_gemv_multi_workspace_size)")
+    _check(load().exl3_gemv_multi(arr, len(layers), m, _dev(workspace, torch.uint8, "workspace"),
+                                  workspace.numel(), _stream(stream)), "exl3_gemv_multi")
+    return ys
+
+
+class GemvMulti:
+    """A prepared exl3_gemv_multi call: the descriptor array is built once, so
+    repeated calls (a decode loop) cost only the C call.  `layers` as for
+    exl3_gemv_multi; the tensors must stay alive and in place."""
+
+    def __init__(self, layers):
+        self.m = layers[0][0].shape[0]
+        self.count = len(layers)
+        self._arr, self.ys = _linear_array(layers, self.m)
+        self.workspace_size = int(load().exl3_gemv_multi_workspace_size(self._arr, self.count, self.m))
+
+    def __call__(self, workspace, stream=None):
+        _check(load().exl3_gemv_multi(self._arr, self.count, self.m, _dev(workspace, torch.uint8, "workspace"),
+                                      workspace.numel(), _stream(stream)), "exl3_gemv_multi")
+        return self.ys
 
 
 def exl3_gemv_noalloc_max_scratch():
