@@ -44,16 +44,6 @@ __device__ __forceinline__ void grid_dep_launch()
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
 }
 
-// ------------------------------------------------------------ bit stream ---
-
-// Words are stored little-endian, the bit string is big-endian per word: the
-// stream order of the bytes of an aligned 32-bit load b0 b1 b2 b3 is
-// b1 b0 b3 b2.  Returns the 32 stream bits with the earliest bit at bit 31.
-__device__ __forceinline__ uint32_t be32(uint32_t raw)
-{
-    return __byte_perm(raw, 0u, 0x1032);
-}
-
 // ------------------------------------------------------------ tile rows ---
 //
 // A tile row holds 16 weights = 16K bits = exactly K words, so row r starts at
