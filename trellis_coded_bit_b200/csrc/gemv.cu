@@ -86,8 +86,10 @@ struct GemvRotLayer {
     int64_t job_begin;  // first job of this layer
 };
 
+constexpr int kGemvRotMaxLayers = 32;  // one rotation launch may serve several main launches
+
 struct GemvRotParams {
-    GemvRotLayer L[kGemvMaxLayers];
+    GemvRotLayer L[kGemvRotMaxLayers];
     int count, m;
     int64_t jobs;
 };
@@ -689,10 +691,41 @@ static exl3_status launch_gemv_k(const GemvParams &p, int K, int smem, cudaStrea
     }
 }
 
-// One launch pair (rotation, main kernel) over up to kGemvMaxLayers layers of
-// the same K, with the workspace region `ws` laid out by gemv_group_plan.
+// Launches the rotation kernel over `count` (<= kGemvRotMaxLayers) layers:
+// layer l's records go to recs[l].
+static exl3_status launch_rotation(const exl3_linear *const *layers, unsigned char *const *recs, int count,
+                                   int64_t m, cudaStream_t stream)
+{
+    const int sms = num_sms();
+    GemvRotParams rp;
+    rp.count = count;
+    rp.m = (int)m;
+    int64_t jobs = 0;
+    const int quads = rec_quads((int)m, 0) + rec_quads((int)m, 1);
+    for (int l = 0; l < count; ++l) {
+        rp.L[l].x = (const __half *)layers[l]->x;
+        rp.L[l].suh = (const __half *)layers[l]->suh;
+        rp.L[l].recs = recs[l];
+        rp.L[l].k = (int)layers[l]->k;
+        rp.L[l].job_begin = jobs;
+        jobs += (int64_t)quads * (layers[l]->k / 128);
+    }
+    rp.jobs = jobs;
+    int64_t rgrid = (jobs + 7) / 8;
+    if (rgrid > 4 * (int64_t)sms)
+        rgrid = 4 * (int64_t)sms;
+    if (rgrid < 1)
+        rgrid = 1;
+    if (launch_kernel(gemv_rotate_kernel, dim3((unsigned)rgrid), dim3(256), 0, stream, rp) != cudaSuccess)
+        return EXL3_ERR_CUDA;
+    return launch_status();
+}
+
+// The main launch over up to kGemvMaxLayers layers of the same K, with the
+// workspace region `ws` laid out by gemv_group_plan; with `rotate` it first
+// launches the rotation for them (else their records are already in place).
 static exl3_status run_gemv_group(const exl3_linear *const *layers, int count, int64_t m, int K,
-                                  unsigned char *ws, size_t ws_bytes, cudaStream_t stream)
+                                  unsigned char *ws, size_t ws_bytes, cudaStream_t stream, bool rotate = true)
 {
     const int sms = num_sms();
     int64_t k[kGemvMaxLayers], n[kGemvMaxLayers];
@@ -704,29 +737,14 @@ static exl3_status run_gemv_group(const exl3_linear *const *layers, int count, i
     if (!ws || !aligned16(ws) || ws_bytes < pl.total)
         return EXL3_ERR_WORKSPACE;
 
-    // rotation -> records
-    GemvRotParams rp;
-    rp.count = count;
-    rp.m = (int)m;
-    int64_t jobs = 0;
-    const int quads = rec_quads((int)m, 0) + rec_quads((int)m, 1);
-    for (int l = 0; l < count; ++l) {
-        rp.L[l].x = (const __half *)layers[l]->x;
-        rp.L[l].suh = (const __half *)layers[l]->suh;
-        rp.L[l].recs = ws + pl.recs[l];
-        rp.L[l].k = (int)k[l];
-        rp.L[l].job_begin = jobs;
-        jobs += (int64_t)quads * (k[l] / 128);
+    if (rotate) {
+        unsigned char *recs[kGemvMaxLayers];
+        for (int l = 0; l < count; ++l)
+            recs[l] = ws + pl.recs[l];
+        const exl3_status rs = launch_rotation(layers, recs, count, m, stream);
+        if (rs != EXL3_OK)
+            return rs;
     }
-    rp.jobs = jobs;
-    int64_t rgrid = (jobs + 7) / 8;
-    if (rgrid > 4 * (int64_t)sms)
-        rgrid = 4 * (int64_t)sms;
-    if (rgrid < 1)
-        rgrid = 1;
-    if (launch_kernel(gemv_rotate_kernel, dim3((unsigned)rgrid), dim3(256), 0, stream, rp) != cudaSuccess ||
-        launch_status() != EXL3_OK)
-        return EXL3_ERR_CUDA;
 
     GemvParams p;
     p.count = count;
@@ -862,9 +880,40 @@ extern "C" exl3_status exl3_gemv_multi(const exl3_linear *layers, int count, int
     if (!workspace || !aligned16(workspace) || workspace_bytes < exl3_gemv_multi_workspace_size(layers, count, m))
         return EXL3_ERR_WORKSPACE;
     unsigned char *ws = (unsigned char *)workspace;
+    cudaStream_t s = (cudaStream_t)stream;
+    // every layer's rotation first, in launches of up to kGemvRotMaxLayers
+    // layers, then one main launch per group reading its records
+    const int sms = num_sms();
+    const exl3_linear *rl[kGemvRotMaxLayers];
+    unsigned char *rr[kGemvRotMaxLayers];
+    int nr = 0;
+    exl3_status st2 = for_each_gemv_group(
+        layers, count, m, [&](const exl3_linear *const *grp, int cnt, int K, size_t off, size_t) {
+            int64_t k[kGemvMaxLayers], n[kGemvMaxLayers];
+            for (int l = 0; l < cnt; ++l) {
+                k[l] = grp[l]->k;
+                n[l] = grp[l]->n;
+            }
+            const GemvGroupPlan pl = gemv_group_plan(k, n, cnt, m, K, sms);
+            for (int l = 0; l < cnt; ++l) {
+                rl[nr] = grp[l];
+                rr[nr] = ws + off + pl.recs[l];
+                if (++nr == kGemvRotMaxLayers) {
+                    const exl3_status rs = launch_rotation(rl, rr, nr, m, s);
+                    if (rs != EXL3_OK)
+                        return rs;
+                    nr = 0;
+                }
+            }
+            return EXL3_OK;
+        });
+    if (st2 == EXL3_OK && nr > 0)
+        st2 = launch_rotation(rl, rr, nr, m, s);
+    if (st2 != EXL3_OK)
+        return st2;
     return for_each_gemv_group(layers, count, m,
                                [&](const exl3_linear *const *grp, int cnt, int K, size_t off, size_t bytes) {
-                                   return run_gemv_group(grp, cnt, m, K, ws + off, bytes, (cudaStream_t)stream);
+                                   return run_gemv_group(grp, cnt, m, K, ws + off, bytes, s, false);
                                });
 }
 
