@@ -122,10 +122,12 @@ exl3_status exl3_gemv(const void *x, const uint16_t *trellis, const void *suh, c
  * a decoder step runs many such layers back to back.)
  *   layers    HOST array of `count` descriptors (copied during the call; the
  *             pointers in it are device memory, laid out as for exl3_gemv).
- *   count     1 .. any; layers are grouped by K and each group (up to 16
- *             layers) runs as one rotation launch plus one persistent launch
- *             whose CTAs share out the group's work units evenly, so the
- *             fixed cost of a launch is paid once per group, not per layer.
+ *   count     1 .. any; every 32 layers (in call order, any mix of K) run
+ *             as one rotation launch plus one persistent launch, so the fixed
+ *             cost of a launch is paid once, not per layer or per K.  The
+ *             persistent launch splits its CTAs into one group per K (in
+ *             proportion to the group's estimated cost), and a group's CTAs
+ *             share out its work units evenly.
  *   workspace at least exl3_gemv_multi_workspace_size bytes, zero-filled
  *             once after allocation, not shared by concurrent calls.
  * Layers must not write one another's inputs (x, trellis, suh, svh).  Results

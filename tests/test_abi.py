@@ -131,7 +131,13 @@ def test_gemv_multi_argument_errors_and_sizes():
 
     one = size([good])
     assert 256 <= one <= lib.exl3_gemv_workspace_size(1, 256, 256, 4)
-    # layers of two K values run as two launches, each with its own region
-    two_k = size([good, (A, B, C, D, E, 512, 1024, 2)])
-    assert two_k >= one + size([(A, B, C, D, E, 512, 1024, 2)])
+    # layers of any mix of K share one launch: one region holding both layers'
+    # activation blocks (k/16 x 512 bytes each) besides the status word
+    other = (A, B, C, D, E, 512, 1024, 2)
+    two_k = size([good, other])
+    assert two_k >= 256 + (256 // 16 + 512 // 16) * 512
+    # more than 32 layers need a second launch, with a region of its own after
+    # the first launch's
+    many = [good] * 33
+    assert size(many) >= size([good] * 32) + size([good])
     assert size([(A, B, C, D, E, 200, 256, 4)]) == 0

@@ -66,7 +66,8 @@ def test_multi_decode_set_matches_oracle_and_single_calls():
 
 
 def test_multi_more_layers_than_one_launch_takes():
-    layers = [inputs.make_layer(2, 256, 256, 2, seed=8500 + i) for i in range(18)]
+    # one launch takes up to 32 layers; 34 of mixed K run as two launches
+    layers = [inputs.make_layer(2, 256, 256, 2 + i % 3, seed=8500 + i) for i in range(34)]
     ys, _, _ = run_multi(layers)
     for L, y in zip(layers, ys):
         check(L, y)

@@ -6,34 +6,37 @@
 // B200 design (the pages' consumer-GPU GEMV is prior art, not copied):
 //   * Two launches.  A rotation kernel computes x' = H(x .* suh)/sqrt(128)
 //     (fp32 butterflies, fp16 result) and writes it into the workspace as
-//     tensor-core A-fragment records (see below).  The main kernel then has
+//     tensor-core B-fragment activation blocks (see below).  The main kernel then has
 //     no prologue: every warp starts streaming weights at once.
-//   * The main kernel is persistent, "stream-K" balanced: the work units are
-//     (128-column block, tile row of 16 input channels) pairs in column-block
-//     order, and CTA c owns the contiguous range [cU/G, (c+1)U/G) -- every
-//     CTA gets the same amount of work, whatever the shape.  A range is cut
-//     into segments at column-block boundaries; inside a segment the 8 warps
-//     take tile rows w, w+8, ...; at a segment end the warps' partial sums
-//     meet in shared memory (one barrier) and either finish the column block
-//     (output rotation, svh, fp16 y) or go to the workspace, where the last
-//     segment to arrive on the block's counter (atomic ticket, no spinning)
-//     sums all segments in segment order (deterministic) and finishes it.
-//   * Lane (g, t) owns tile g of the column block and, in each of 4 row
-//     groups q, the whole tile row rho(q, t) (16 weights): rows are ordered
-//     so that all lanes of a group share the row parity, which makes every
-//     bit-window operation a compile-time byte permute (see row_states).
-//     Loads go straight from HBM into registers in this fragment order
-//     (read-only path, 8/16-byte vectors where aligned), one unit ahead of
-//     the math and across segment boundaries.
-//   * The MAC runs on the tensor cores (mma.sync m16n8k16, fp32 accumulate):
-//     a codebook word's two fp16 halves form a pair of k slots in B and the
-//     activation is duplicated over that pair in A, so the tensor core forms
-//     x*(hi + lo) exactly in fp32 (the fp16 rounding of hi + lo that defines
-//     W_hat is skipped: at most half an fp16 ulp per weight, far inside the
-//     output tolerance).  Weights 2j, 2j+1 of a lane's row feed MMA j (k
-//     pairs t and t+4); A rows are (batch, column parity) with zeros
-//     elsewhere, so parities never mix.  Batch rows 0..7 per group, two
-//     groups for m > 8 (one decode feeds both).
+//   * The main kernel is persistent and "stream-K" balanced at warp level:
+//     the work units are (layer, 128-column block, tile row of 16 input
+//     channels), numbered consecutively over every layer of the launch (any
+//     mix of K), and warp w of W owns the contiguous range [wU/W, (w+1)U/W)
+//     -- every warp gets the same amount of work, whatever the shapes.  A
+//     range is cut into segments at column-block boundaries.  At a segment end
+//     the warp writes its fp32 partial of the block to the workspace; the last
+//     warp to arrive on the block's counter (atomic ticket, no spinning) sums
+//     the block's partials in a fixed order (deterministic) and finishes it
+//     (output rotation, svh, fp16 y).  Warps never wait for one another, and
+//     one launch serves all the layers of an exl3_gemv_multi call.
+//   * The MAC runs on the tensor cores (mma.sync m16n8k16, fp32 accumulate)
+//     with the WEIGHTS in the A operand: a codebook word's two fp16 halves
+//     form a pair of k slots and the activation is duplicated over that pair
+//     in B, so the tensor core forms x*(hi + lo) exactly in fp32 (the fp16
+//     rounding of hi + lo that defines W_hat is skipped: at most half an fp16
+//     ulp per weight, far inside the output tolerance).  One MMA thus takes
+//     16 output columns x 8 input channels = 128 weights, and its 8 B columns
+//     are 8 batches: at m = 1 the tensor pipe does half the work it would
+//     with the weights in B.
+//   * Lane (g, t) owns tile g of the 128-column block and, in k-step ks, the
+//     two adjacent tile rows 8ks + 2t and 8ks + 2t + 1: one contiguous run of
+//     2K + 1 words (with the prefix word) whose 32 bit windows are
+//     compile-time byte permutes (pair_states).  Weight (row 8ks + 2t + p,
+//     column c) goes to A row g + 8(c & 1), k-pair t + 4p of MMA c / 2, so
+//     MMA j accumulates columns 2j and 2j + 1 of every tile of the block.
+//   * Each warp streams its units through its own 3-deep cp.async ring in
+//     shared memory (8 tiles padded against bank conflicts, plus the unit's
+//     activation block), loaded by 16-byte copies spread over the lanes.
 //   * With EXL3_LAUNCH_PDL the main kernel requests its first weights before
 //     it waits for the rotation kernel (griddepcontrol).
 #include <cuda_fp16.h>
@@ -46,47 +49,33 @@ namespace exl3 {
 constexpr int kGemvWarps = 8;
 constexpr int kGemvThreads = 32 * kGemvWarps;
 
-// Activation records, in MMA A-fragment register order.  For batch group mg
-// (batches 8mg..8mg+7), quad ba (batches 8mg+ba and 8mg+ba+4) and A-row
-// parity p, a 16-byte record holds the lane's {a0, a1, a2, a3}:
-//   p = 0: {x(8mg+ba), x(8mg+ba+4), 0, 0}     p = 1: {0, 0, x(8mg+ba), x(8mg+ba+4)}
-// with x the rotated activation duplicated in both fp16 halves (a batch
-// >= m is zero).  Each input channel has rec_slots_for(MG) = 8 MG slots, slot
-// 8mg + 2ba + p, record (kk, slot) at recs + (kk * 8 MG + slot) * 16.  Only
-// quads holding a batch < m are written: a record of an absent quad feeds only
-// A rows of absent batches, whose accumulator rows are never stored, so
-// whatever it holds is harmless.
-__host__ __device__ inline int rec_quads(int m, int mg)
-{
-    const int q = m - 8 * mg;
-    return q <= 0 ? 0 : (q < 4 ? q : 4);
-}
-
-__host__ __device__ constexpr int rec_slots_for(int MG)
-{
-    return 8 * MG;
-}
+// Activation blocks, in MMA B-fragment register order.  For tile row tr
+// (input channels 16tr .. 16tr+15) and batch group mg (batches 8mg .. 8mg+7)
+// a 512-byte block; its 8-byte entry (ks, g, t) at ks*256 + g*32 + t*8 holds
+// channels 16tr + 8ks + 2t and 16tr + 8ks + 2t + 1 of batch 8mg + g, each an
+// fp16 duplicated into both halves of a 32-bit word: exactly the (b0, b1)
+// that lane (g, t) feeds the MMA in k-step ks.  Block (tr, mg) sits at
+// (tr * MG + mg) * 512.  Only batches < m are written and copied; the ring's
+// entries of absent batches are zero (they feed only B columns whose
+// accumulators are never stored).
+__host__ __device__ constexpr int kGemvActBlock = 512;
 
 __host__ __device__ inline int gemv_mg(int64_t m)
 {
     return m > 8 ? 2 : 1;
 }
 
-// Up to kGemvMaxLayers layers (same K and m) share one launch; their work
-// units and column blocks are numbered consecutively across the layers.
-constexpr int kGemvMaxLayers = 16;
-
 // ------------------------------------------------------ rotation kernel ---
 
 struct GemvRotLayer {
     const __half *x;
     const __half *suh;
-    unsigned char *recs;
+    unsigned char *acts;
     int k;
     int64_t job_begin;  // first job of this layer
 };
 
-constexpr int kGemvRotMaxLayers = 32;  // one rotation launch may serve several main launches
+constexpr int kGemvRotMaxLayers = 32;  // at least the main launch's layer limit
 
 struct GemvRotParams {
     GemvRotLayer L[kGemvRotMaxLayers];
@@ -94,16 +83,15 @@ struct GemvRotParams {
     int64_t jobs;
 };
 
-// One warp per (layer, quad, 128-channel block): rotates the quad's one or
-// two batches and writes both parity records of each channel.
+// One warp per (layer, batch, 128-channel block): lane l rotates channels
+// 4l .. 4l+3 and writes them as one 16-byte piece of the activation blocks.
 __global__ void __launch_bounds__(256) gemv_rotate_kernel(const GemvRotParams rp)
 {
     grid_dep_wait();    // x may come from the preceding kernel
     grid_dep_launch();  // the main kernel may start streaming weights meanwhile
     const int lane = threadIdx.x & 31;
     const int m = rp.m;
-    const int slots = rec_slots_for(gemv_mg(m));
-    const int q0 = rec_quads(m, 0);
+    const int MG = gemv_mg(m);
     const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
     const float s128 = 0.08838834764831845f;
     int l = 0;
@@ -113,80 +101,101 @@ __global__ void __launch_bounds__(256) gemv_rotate_kernel(const GemvRotParams rp
         const GemvRotLayer &L = rp.L[l];
         const int k = L.k, nblk = k / 128;
         const int64_t lj = job - L.job_begin;
-        const int qd = (int)(lj / nblk), blk = (int)(lj - (int64_t)qd * nblk);
-        const int mg = qd >= q0 ? 1 : 0, ba = qd - mg * q0;
-        const int b0 = 8 * mg + ba, b1 = b0 + 4;
+        const int b = (int)(lj / nblk), blk = (int)(lj - (int64_t)b * nblk);
         const int c = blk * 128 + lane * 4;
         const uint2 sr = *reinterpret_cast<const uint2 *>(L.suh + c);
-        const uint2 r0 = *reinterpret_cast<const uint2 *>(L.x + (int64_t)b0 * k + c);
-        uint2 r1 = make_uint2(0u, 0u);
-        if (b1 < m)
-            r1 = *reinterpret_cast<const uint2 *>(L.x + (int64_t)b1 * k + c);
+        const uint2 r0 = *reinterpret_cast<const uint2 *>(L.x + (int64_t)b * k + c);
         const __half2 *sv = reinterpret_cast<const __half2 *>(&sr);
         const __half2 *x0 = reinterpret_cast<const __half2 *>(&r0);
-        const __half2 *x1 = reinterpret_cast<const __half2 *>(&r1);
-        float v0[4] = {__low2float(x0[0]) * __low2float(sv[0]), __high2float(x0[0]) * __high2float(sv[0]),
-                       __low2float(x0[1]) * __low2float(sv[1]), __high2float(x0[1]) * __high2float(sv[1])};
-        float v1[4] = {__low2float(x1[0]) * __low2float(sv[0]), __high2float(x1[0]) * __high2float(sv[0]),
-                       __low2float(x1[1]) * __low2float(sv[1]), __high2float(x1[1]) * __high2float(sv[1])};
-        warp_fwht128(v0);
-        warp_fwht128(v1);
+        float v[4] = {__low2float(x0[0]) * __low2float(sv[0]), __high2float(x0[0]) * __high2float(sv[0]),
+                      __low2float(x0[1]) * __low2float(sv[1]), __high2float(x0[1]) * __high2float(sv[1])};
+        warp_fwht128(v);
+        uint32_t d[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const uint32_t h0 = (uint32_t)__half_as_ushort(__float2half_rn(v0[e] * s128));
-            const uint32_t h1 = b1 < m ? (uint32_t)__half_as_ushort(__float2half_rn(v1[e] * s128)) : 0u;
-            const uint32_t d0 = h0 | (h0 << 16), d1 = h1 | (h1 << 16);
-            uint4 *rec = reinterpret_cast<uint4 *>(L.recs + ((int64_t)(c + e) * slots + 8 * mg + 2 * ba) * 16);
-            rec[0] = make_uint4(d0, d1, 0u, 0u);  // even A rows
-            rec[1] = make_uint4(0u, 0u, d0, d1);  // odd A rows
+            const uint32_t h = (uint32_t)__half_as_ushort(__float2half_rn(v[e] * s128));
+            d[e] = h | (h << 16);
         }
+        // channels c .. c+3: tile row c / 16, rows r .. r+3 with r = c % 16
+        // (r = 8ks + 2t0, t0 even): entries (ks, g, t0) and (ks, g, t0 + 1)
+        const int tr = c >> 4, r = c & 15;
+        const int mg = b >> 3, g = b & 7;
+        unsigned char *dst = L.acts + ((int64_t)tr * MG + mg) * kGemvActBlock + (r >> 3) * 256 + g * 32 +
+                             ((r & 7) >> 1) * 8;
+        *reinterpret_cast<uint4 *>(dst) = make_uint4(d[0], d[1], d[2], d[3]);
     }
 }
 
 // ---------------------------------------------------------- main kernel ---
 
-// One layer of a launch.  Global unit u of the layer is unit_begin + cb * TR
-// + tr (column block cb, tile row tr); its column blocks are the launch's
-// column blocks cb_begin .. cb_begin + n/128 - 1.
+// One launch covers up to kGemvMaxLayers layers with the same m and any mix
+// of K.  The layers are grouped by K; each group gets its own share of the
+// grid's CTAs (in proportion to its estimated cost), so that every CTA runs
+// the decode compiled for one K.  Within a group the work units -- (layer,
+// 128-column block, tile row) -- are numbered consecutively: layer by layer,
+// column block by column block, tile row by tile row.
+constexpr int kGemvMaxLayers = 32;
+
 struct GemvLayer {
-    const unsigned char *trellis;
+    const unsigned char *trellis;  // uint16 [k/16][n/16][16K]
     const __half *svh;
     __half *y;
-    const unsigned char *recs;
-    float *partials;     // [n/128][max_seg][m][128]
-    uint32_t *counters;  // [n/128]
-    int64_t unit_begin;
-    int n, tr_count, cb_begin, max_seg;
+    const unsigned char *acts;  // activation blocks [k/16][MG][512 B]
+    float *partials;            // [n/128][max_seg][m][128]
+    uint32_t *counters;         // [n/128]
+    int64_t unit_begin;         // the layer's first unit within its group
+    int n, tr_count, max_seg;
+    int cb_begin;               // the layer's first column block within its group
+};
+
+// A group: the layers [l_begin, l_end) of one K, run by the CTAs
+// [cta_begin, cta_begin + ctas) over its `units` units.
+struct GemvGroup {
+    int64_t units;
+    int K, l_begin, l_end, cta_begin, ctas;
+};
+
+// Multipliers the window extraction uses in place of shifts, passed in as
+// launch parameters so that they stay opaque registers: a multiply by a
+// register runs on the FMA pipe (IMAD), which the decode leaves half idle,
+// while shifts and byte permutes compete with the codebook's LOP3 for the
+// ALU pipe.  pow2[i] = 2^i, hi16 = 2^16 (mul.hi by it is a right shift by 16).
+struct GemvMults {
+    uint32_t pow2[8];
+    uint32_t hi16;
 };
 
 struct GemvParams {
     GemvLayer L[kGemvMaxLayers];
-    int count, m, ctas;
-    int64_t units;  // all layers' units
+    GemvGroup grp[8];
+    int ngroups, m;
     Codebook cb;
+    GemvMults mu;
 };
 
-// Per-warp shared-memory ring: each stage holds one unit -- the 8 tiles of a
-// tile row (each padded to 32K + 16 bytes, which spreads the lanes' row reads
-// over the banks) and that tile row's 16 x 8MG activation records.  The
-// layout is a compile-time function of K and MG, so every shared-memory
-// access of the inner loop is a lane pointer plus an immediate offset.
-template <int K, int MG>
-struct GemvStage {
-    static constexpr int kTileStride = 32 * K + 16;
-    static constexpr int kTileBytes = 8 * kTileStride;
-    static constexpr int kSlots = rec_slots_for(MG);
-    static constexpr int kRecRowBytes = 16 * kSlots * 16;  // records of one tile row
-    static constexpr int kBytes = (kTileBytes + kRecRowBytes + 127) & ~127;
-};
-
-__host__ __device__ inline int gemv_stage_bytes(int K, int MG)
+// Per-warp shared-memory ring of kGemvDepth stages; a stage holds one unit:
+// the tile row's activation blocks (MG x 512 bytes, at the stage start, so
+// their place does not depend on K) and then the unit's 8 tiles, each padded
+// to 32K + pad bytes so that the lanes' run reads spread over the banks (the
+// pad per K minimises the modelled shared-memory wavefronts of those reads).
+// Within a stage every offset is a compile-time function of K and MG, so the
+// inner loop addresses shared memory as a lane pointer plus immediates.
+__host__ __device__ constexpr int gemv_tile_pad(int K)
 {
-    const int tiles = 8 * (32 * K + 16), recs = 16 * rec_slots_for(MG) * 16;
-    return (tiles + recs + 127) & ~127;
+    return K == 4 ? 64 : ((K == 2 || K == 6) ? 32 : 16);
 }
 
-constexpr int kGemvDepth = 3;  // units in flight per warp (one consumed, two loading)
+__host__ __device__ constexpr int gemv_tile_stride(int K)
+{
+    return 32 * K + gemv_tile_pad(K);
+}
+
+__host__ __device__ constexpr int gemv_stage_bytes(int K, int MG)
+{
+    return (MG * kGemvActBlock + 8 * gemv_tile_stride(K) + 127) & ~127;
+}
+
+constexpr int kGemvDepth = 3;  // units in flight per warp (one consumed, the rest loading)
 
 __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc)
 {
@@ -205,98 +214,156 @@ __device__ __forceinline__ void cp_async_wait()
     asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
-// Lane (g, t) owns tile g of the unit and, in row group q, the tile row
-// rho(q, t) = 2t + c(q) with c(q) = 8(q & 1) + (q >> 1): groups 0, 1 take
-// the even rows, groups 2, 3 the odd ones, so a group's lanes share the row
-// parity (compile-time bit windows).  Row rho starts at word rho K; its
-// prefix word (rho K - 1) wraps to the tile's last word for rho = 0.
+// The 32 states of a row pair from its run of words.  R[0] holds the prefix
+// word in its upper half, R[i] (i = 1..K) holds the pair's words 2i - 2
+// (lower half) and 2i - 1 (upper half).  Counting stream positions from the
+// prefix word W'[0] (W'[i] = positions 16i .. 16i + 15; W'[2i-1] is R[i]'s
+// lower half, W'[2i] its upper half), weight jj (row jj / 16, column jj % 16)
+// has the window ending at position e = 16 + (jj + 1) K.  When e is a
+// multiple of 16 the window is the word W'[e/16 - 1]; otherwise it lies in
+// V = W'[a-1]:W'[a] (a = e / 16, as one big-endian 32-bit value) shifted
+// right by c = 16 - e % 16, and is one byte permute with zero fill of V or of
+// V pre-shifted by c % 8.  All selectors are compile-time constants, and the
+// V values and their shifted copies are shared between windows.
 template <int K>
-__host__ __device__ constexpr int gemv_row_imm(int q)
+__device__ __forceinline__ void pair_states(const uint32_t (&R)[K + 1], uint32_t (&s)[32], const GemvMults &mu)
 {
-    return 4 * (((8 * (q & 1) + (q >> 1)) * K - 1) >> 1);  // floor, -4 for c(q) = 0
+#pragma unroll
+    for (int jj = 0; jj < 32; ++jj) {
+        const int e = 16 + (jj + 1) * K;
+        const int a = e >> 4, rb = e & 15;
+        if (rb == 0) {
+            const int w = a - 1;
+#if GEMV_WORD_HI_IMAD
+            s[jj] = (w & 1) ? __byte_perm(R[(w + 1) >> 1], 0u, 0x4410u) : __umulhi(R[w >> 1], mu.hi16);
+#else
+            s[jj] = (w & 1) ? __byte_perm(R[(w + 1) >> 1], 0u, 0x4410u) : __byte_perm(R[w >> 1], 0u, 0x4432u);
+#endif
+        } else {
+            const uint32_t v = (a & 1) ? __byte_perm(R[(a - 1) >> 1], R[(a + 1) >> 1], 0x3254u)
+                                       : __byte_perm(R[a >> 1], 0u, 0x1032u);
+            const int c = 16 - rb, r = c & 7, cb = c >> 3;
+            if (r == 0) {
+                s[jj] = __byte_perm(v, 0u, 0x4400u | ((uint32_t)(cb + 1) << 4) | (uint32_t)cb);
+            } else {
+                // bits [c, c + 16) of v are bits [8(cb + 1), 8(cb + 1) + 16) of
+                // v * 2^(8 - r); the bits shifted out lie above the window
+                const uint32_t vs = v * mu.pow2[8 - r];
+                s[jj] = __byte_perm(vs, 0u, 0x4400u | ((uint32_t)(cb + 2) << 4) | (uint32_t)(cb + 1));
+            }
+        }
+    }
 }
 
-// The lane's base pointers into its ring (stage 0): row words, the q = 0
-// prefix word (the wrap lane differs), activation records.
+// The lane's pointers into its ring's stage 0: its tile's k-step-0 run (word
+// tK), its k-step-0 prefix word (the tile's last word for t = 0: the
+// tail-biting wrap), and its activation entry.
 struct GemvLanePtrs {
-    const unsigned char *row, *pre0, *rec;
+    const unsigned char *run, *pre0, *act;
 };
 
-// Loads the words of tile row rho(q, t) of stage S: raw[0] the prefix word,
-// then the row's words, as wide as the row's alignment allows.
-template <int K, int MG, int S, int q, int N>
-__device__ __forceinline__ void load_row_q(const GemvLanePtrs &lp, uint32_t (&raw)[N])
+// Loads the words of the lane's row pair of k-step KS in the stage at byte
+// offset OFF: R[0] the prefix word, R[1..K] the pair's 2K words, as wide as
+// the run's alignment allows (4tK bytes into a 16-byte aligned tile: 16 bytes
+// for K % 4 == 0, 8 for even K, else 4).
+template <int K, int KS, int OFF>
+__device__ __forceinline__ void load_pair(const GemvLanePtrs &lp, uint32_t (&R)[K + 1])
 {
-    using St = GemvStage<K, MG>;
-    constexpr int PAR = q >> 1;
-    constexpr int P = RowSpan<K, PAR>::P;
-    constexpr int N32 = RowSpan<K, PAR>::N32;
-    constexpr int off = S * St::kBytes + gemv_row_imm<K>(q);
-    const unsigned char *row = lp.row + off;
-    raw[0] = (q == 0) ? *reinterpret_cast<const uint32_t *>(lp.pre0 + S * St::kBytes)
-                      : *reinterpret_cast<const uint32_t *>(row - 4);
-    if constexpr (K == 4 && P == 1) {
-        const uint2 v = *reinterpret_cast<const uint2 *>(row);
-        raw[1] = v.x;
-        raw[2] = v.y;
-    } else if constexpr (K == 8 && P == 1) {
-        const uint4 v = *reinterpret_cast<const uint4 *>(row);
-        raw[1] = v.x;
-        raw[2] = v.y;
-        raw[3] = v.z;
-        raw[4] = v.w;
+    const unsigned char *run = lp.run + OFF + KS * 16 * K;
+    R[0] = KS == 0 ? *reinterpret_cast<const uint32_t *>(lp.pre0 + OFF) : *reinterpret_cast<const uint32_t *>(run - 4);
+    if constexpr (K % 4 == 0) {
+#pragma unroll
+        for (int i = 0; i < K / 4; ++i) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(run + 16 * i);
+            R[4 * i + 1] = v.x;
+            R[4 * i + 2] = v.y;
+            R[4 * i + 3] = v.z;
+            R[4 * i + 4] = v.w;
+        }
+    } else if constexpr (K % 2 == 0) {
+#pragma unroll
+        for (int i = 0; i < K / 2; ++i) {
+            const uint2 v = *reinterpret_cast<const uint2 *>(run + 8 * i);
+            R[2 * i + 1] = v.x;
+            R[2 * i + 2] = v.y;
+        }
     } else {
 #pragma unroll
-        for (int i = 1; i < N32; ++i)
-            raw[i] = *reinterpret_cast<const uint32_t *>(row + 4 * (i - 1));
+        for (int i = 0; i < K; ++i)
+            R[i + 1] = *reinterpret_cast<const uint32_t *>(run + 4 * i);
     }
 }
 
-template <int K, int MG, int S, int q>
-__device__ __forceinline__ void mac_row(const GemvLanePtrs &lp, const Codebook &cb, float (&acc)[MG][8][4])
+// One unit held in ring stage ST: for each k-step decode the lane's row pair
+// (32 weights) and run the 8 MMAs (per batch group) that consume it.
+template <int K, int MG, int ST>
+__device__ __forceinline__ void mac_unit(const GemvLanePtrs &lp, const Codebook &cb, const GemvMults &mu,
+                                         float (&acc)[MG][8][4])
 {
-    using St = GemvStage<K, MG>;
-    constexpr int PAR = q >> 1;
-    constexpr int cq = 8 * (q & 1) + (q >> 1);
-    uint32_t A[MG][4];
+    constexpr int OFF = ST * gemv_stage_bytes(K, MG);
 #pragma unroll
-    for (int mg = 0; mg < MG; ++mg) {
-        const uint4 r = *reinterpret_cast<const uint4 *>(lp.rec + S * St::kBytes + cq * St::kSlots * 16 + mg * 128);
-        A[mg][0] = r.x;
-        A[mg][1] = r.y;
-        A[mg][2] = r.z;
-        A[mg][3] = r.w;
-    }
-    uint32_t raw[RowSpan<K, PAR>::N32];
-    load_row_q<K, MG, S, q>(lp, raw);
-    uint32_t st[16];
-    row_states<K, RowSpan<K, PAR>::P>(raw, st);
+    for (int ks = 0; ks < 2; ++ks) {
+        uint32_t B[MG][2];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const uint32_t b0 = codebook_word(st[2 * j], cb);
-        const uint32_t b1 = codebook_word(st[2 * j + 1], cb);
+        for (int mg = 0; mg < MG; ++mg) {
+            const uint2 b = *reinterpret_cast<const uint2 *>(lp.act + OFF + ks * 256 + mg * kGemvActBlock);
+            B[mg][0] = b.x;
+            B[mg][1] = b.y;
+        }
+        uint32_t R[K + 1];
+        if (ks == 0)
+            load_pair<K, 0, OFF>(lp, R);
+        else
+            load_pair<K, 1, OFF>(lp, R);
+        uint32_t st[32];
+        pair_states<K>(R, st, mu);
 #pragma unroll
-        for (int mg = 0; mg < MG; ++mg)
-            mma_16816(acc[mg][j], A[mg], b0, b1);
+        for (int j = 0; j < 8; ++j) {
+            const uint32_t a[4] = {codebook_word(st[2 * j], cb), codebook_word(st[2 * j + 1], cb),
+                                   codebook_word(st[16 + 2 * j], cb), codebook_word(st[17 + 2 * j], cb)};
+#pragma unroll
+            for (int mg = 0; mg < MG; ++mg)
+                mma_16816(acc[mg][j], a, B[mg][0], B[mg][1]);
+        }
     }
 }
 
-template <int K, int MG, int S>
-__device__ __forceinline__ void mac_stage(const GemvLanePtrs &lp, const Codebook &cb, float (&acc)[MG][8][4])
+// mac_unit for a stage index known only at run time (one compiled copy per
+// stage, so every shared-memory offset stays an immediate).
+template <int K, int MG, int ST>
+__device__ __forceinline__ void mac_unit_at(int st, const GemvLanePtrs &lp, const Codebook &cb,
+                                            const GemvMults &mu, float (&acc)[MG][8][4])
 {
-    mac_row<K, MG, S, 0>(lp, cb, acc);
-    mac_row<K, MG, S, 1>(lp, cb, acc);
-    mac_row<K, MG, S, 2>(lp, cb, acc);
-    mac_row<K, MG, S, 3>(lp, cb, acc);
+    if constexpr (ST + 1 < kGemvDepth) {
+        if (st == ST)
+            mac_unit<K, MG, ST>(lp, cb, mu, acc);
+        else
+            mac_unit_at<K, MG, ST + 1>(st, lp, cb, mu, acc);
+    } else {
+        mac_unit<K, MG, ST>(lp, cb, mu, acc);
+    }
 }
 
 // CTA owning unit u: the largest c with floor(c U / G) <= u.
-__device__ __forceinline__ int owner_cta(int64_t u, int64_t U, int G)
+__host__ __device__ inline int64_t gemv_owner_cta(int64_t u, int64_t U, int64_t G)
 {
-    return (int)(((u + 1) * G - 1) / U);
+    return ((u + 1) * G - 1) / U;
 }
 
-// Output rotation, svh and fp16 store of one column block's m x 128 y'.
+// Position of unit u of a group: layer l (scanning on from l, within
+// [lb, le)), column block cb within it, tile row tr.
+__device__ __forceinline__ void gemv_locate(const GemvParams &p, int le, int64_t u, int &l, int &cb, int &tr)
+{
+    while (l + 1 < le && u >= p.L[l + 1].unit_begin)
+        ++l;
+    const int64_t lu = u - p.L[l].unit_begin;
+    const int TR = p.L[l].tr_count;
+    cb = (int)(lu / TR);
+    tr = (int)(lu - (int64_t)cb * TR);
+}
+
+// Output rotation, svh and fp16 store of one column block's m x 128 y'
+// (summed in shared memory): a warp per batch row.
 __device__ __forceinline__ void finish_block(const GemvLayer &L, int m, const float *red, int cb, int warp,
                                              int lane)
 {
@@ -319,111 +386,137 @@ __device__ __forceinline__ void finish_block(const GemvLayer &L, int m, const fl
     }
 }
 
-// Position of global unit u: layer l (scanning on from l; always 0 for a
-// single-layer launch), column block cb within it, tile row tr.
-template <bool MULTI>
-__device__ __forceinline__ void gemv_locate(const GemvParams &p, int64_t u, int &l, int &cb, int &tr)
+// The work of one CTA of a K group.  CTA c of the group's G owns the
+// contiguous unit range [cU/G, (c+1)U/G); its 8 warps take units u0 + w,
+// u0 + w + 8, ..., so that a CTA's concurrent loads stay within a few
+// consecutive tile rows.  The range is cut into segments at column-block
+// boundaries; at a segment end the warps' partials meet in shared memory (a
+// CTA barrier) and either finish the block or go to the workspace, where the
+// last segment to arrive (atomic ticket, no spinning) sums all segments in
+// segment order and finishes it.
+template <int K, int MG>
+__device__ __forceinline__ void gemv_cta(const GemvParams &p, const GemvGroup &gp)
 {
-    while (MULTI && l + 1 < p.count && u >= p.L[l + 1].unit_begin)
-        ++l;
-    const int64_t lu = u - p.L[l].unit_begin;
-    const int TR = p.L[l].tr_count;
-    cb = (int)(lu / TR);
-    tr = (int)(lu - (int64_t)cb * TR);
-}
-
-template <int K, int MG, bool MULTI>
-__global__ void __launch_bounds__(kGemvThreads, MG == 1 ? 2 : 1) gemv_kernel(const GemvParams p)
-{
-    using St = GemvStage<K, MG>;
-    constexpr int SB = St::kBytes;
+    constexpr int SB = gemv_stage_bytes(K, MG);
+    constexpr int S = gemv_tile_stride(K);
     constexpr int kTrChunks = (16 * K + 31) / 32;  // 16-byte trellis chunks per lane per unit
-    constexpr int kRecChunks = St::kRecRowBytes / 16 / 32;
     extern __shared__ __align__(128) unsigned char smem[];
     volatile int *flag = reinterpret_cast<volatile int *>(smem);
     const int m = p.m;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    unsigned char *ring = smem + 128 + warp * kGemvDepth * SB;
-    float *red = reinterpret_cast<float *>(smem + 128 + kGemvWarps * kGemvDepth * SB);
-
     const int g = lane >> 2, t = lane & 3;
-    const int64_t U = p.units;
-    const int G = p.ctas;
-    const int64_t u0 = (int64_t)blockIdx.x * U / G, u1 = (int64_t)(blockIdx.x + 1) * U / G;
+    float *red = reinterpret_cast<float *>(smem + 128);
+    unsigned char *ring = smem + 128 + kGemvWarps * m * 128 * 4 + warp * kGemvDepth * SB;
+    const int lb = gp.l_begin, le = gp.l_end;
+    const int64_t U = gp.units;
+    const int64_t G = gp.ctas;
+    const int64_t c = (int64_t)blockIdx.x - gp.cta_begin;
+    const int64_t u0 = c * U / G, u1 = (c + 1) * U / G;
 
-    // lane-constant pointers and copy offsets
     GemvLanePtrs lp;
-    lp.row = ring + g * St::kTileStride + 4 * (t * K + 1);
-    lp.pre0 = t == 0 ? ring + g * St::kTileStride + 4 * (8 * K - 1)  // row 0: the tile's last word
-                     : lp.row + gemv_row_imm<K>(0) - 4;
-    lp.rec = ring + St::kTileBytes + (2 * t * St::kSlots + g) * 16;
+    lp.run = ring + MG * kGemvActBlock + g * S + 4 * t * K;
+    lp.pre0 = t == 0 ? ring + MG * kGemvActBlock + g * S + 4 * (8 * K - 1) : lp.run - 4;
+    lp.act = ring + g * 32 + t * 8;
+    // the lane's trellis chunks (chunk i = lane + 32r of the unit's 16K: tile
+    // i / 2K, 16-byte piece i % 2K) and activation chunks (entry row (ks, g')
+    // with g' = (lane >> 1) & 7, i.e. batch 8 mg + g'; only batches < m)
     unsigned char *tdst[kTrChunks];
 #pragma unroll
     for (int r = 0; r < kTrChunks; ++r) {
-        const int i = lane + 32 * r;  // chunk i: tile i / 2K, 16-byte piece i % 2K
-        tdst[r] = ring + (i / (2 * K)) * St::kTileStride + (i % (2 * K)) * 16;
+        const int i = lane + 32 * r;
+        tdst[r] = ring + MG * kGemvActBlock + (i / (2 * K)) * S + (i % (2 * K)) * 16;
     }
     const bool last_chunk = (16 * K) % 32 == 0 || lane + 32 * (kTrChunks - 1) < 16 * K;
+    bool act_live[MG];
+#pragma unroll
+    for (int mg = 0; mg < MG; ++mg)
+        act_live[mg] = 8 * mg + ((lane >> 1) & 7) < m;
 
-    // this warp's units: u0 + warp, u0 + warp + 8, ... (< u1), as (layer,
-    // column block, tile row) advanced incrementally; the issue iterator runs
-    // kGemvDepth units ahead of consumption
+    // issue iterator (runs kGemvDepth units ahead of consumption): unit iu at
+    // (layer il, column block icb, tile row itr), advancing by 8 units
     int64_t iu = u0 + warp;
-    int il = 0, icb = 0, itr = 0;
-    gemv_locate<MULTI>(p, iu < u1 ? iu : u0, il, icb, itr);
+    int il = lb, icb = 0, itr = 0;
+    gemv_locate(p, le, iu < u1 ? iu : u0, il, icb, itr);
+    int itr_lim = 0, incb = 0;
     int64_t tile_row_bytes = 0;
-    int itr_lim = 0, incb = 0;  // the issue layer's tile rows and column blocks
-    const unsigned char *isrc = nullptr, *irsrc = nullptr;
-    auto point = [&]() {
+    const unsigned char *isrc = nullptr, *iasrc = nullptr;
+    auto enter_block = [&]() {
         const GemvLayer &L = p.L[il];
         itr_lim = L.tr_count;
         incb = L.n >> 7;
-        tile_row_bytes = (int64_t)(L.n >> 4) * 32 * K;  // one tile row of the layer's matrix
-        isrc = L.trellis + itr * tile_row_bytes + (int64_t)icb * 8 * 32 * K + lane * 16;
-        irsrc = L.recs + (int64_t)itr * St::kRecRowBytes + lane * 16;
+        tile_row_bytes = (int64_t)(L.n >> 4) * 32 * K;
+        isrc = L.trellis + itr * tile_row_bytes + (int64_t)icb * 256 * K + lane * 16;
+        iasrc = L.acts + (int64_t)itr * MG * kGemvActBlock + lane * 16;
     };
-    point();
-    int64_t cu = iu;
-    int cl = il, ccb = icb, ctr = itr;  // consumed unit: layer, column block, tile row
-    int cg = p.L[il].cb_begin + icb;    // consumed unit's global column block
-    int ctr_lim = itr_lim, cncb = incb;  // the consumed unit's layer: tile rows, column blocks
-
-    auto issue = [&](int stage) {
-        if (iu < u1) {
-            const int so = stage * SB;
+    if (iu < u1)
+        enter_block();
+    auto copy_acts = [&](int stage, const unsigned char *src) {
 #pragma unroll
-            for (int r = 0; r < kTrChunks; ++r)
-                if (r < kTrChunks - 1 || last_chunk)
-                    cp_async16(tdst[r] + so, isrc + 512 * r);
+        for (int mg = 0; mg < MG; ++mg)
+            if (act_live[mg])
+                cp_async16(ring + stage * SB + mg * kGemvActBlock + lane * 16, src + mg * kGemvActBlock);
+    };
+    // copies the trellis of the issue iterator's unit into `stage`, returns
+    // the unit's activation source (null past the range) and advances
+    auto issue_trellis = [&](int stage) -> const unsigned char * {
+        if (iu >= u1)
+            return nullptr;
+        const unsigned char *asrc = iasrc;
+        const int so = stage * SB;
 #pragma unroll
-            for (int r = 0; r < kRecChunks; ++r)
-                cp_async16(ring + so + St::kTileBytes + (lane + 32 * r) * 16, irsrc + 512 * r);
-            iu += kGemvWarps;
-            itr += kGemvWarps;
-            isrc += kGemvWarps * tile_row_bytes;
-            irsrc += kGemvWarps * St::kRecRowBytes;
-            if (itr >= itr_lim) {  // next column block, perhaps of the next layer (units advance by 8 <= TR)
-                itr -= itr_lim;
-                if (++icb == incb) {
-                    icb = 0;
-                    if (MULTI)
-                        ++il;
-                }
-                if (iu < u1)
-                    point();
+        for (int r = 0; r < kTrChunks; ++r)
+            if (r < kTrChunks - 1 || last_chunk)
+                cp_async16(tdst[r] + so, isrc + 512 * r);
+        iu += kGemvWarps;
+        itr += kGemvWarps;
+        isrc += kGemvWarps * tile_row_bytes;
+        iasrc += kGemvWarps * MG * kGemvActBlock;
+        if (itr >= itr_lim) {  // next column block, perhaps of the next layer (8 <= every TR)
+            itr -= itr_lim;
+            if (++icb == incb) {
+                icb = 0;
+                ++il;
             }
+            if (iu < u1)
+                enter_block();
         }
+        return asrc;
+    };
+    auto issue = [&](int stage) {
+        const unsigned char *asrc = issue_trellis(stage);
+        if (asrc)
+            copy_acts(stage, asrc);
         cp_async_commit();
     };
 
-    // records come from the rotation kernel: wait for it (no-op without PDL)
-    grid_dep_wait();
+    // Prologue: the first kGemvDepth units' weights are requested before the
+    // wait for the rotation kernel (which writes the activation blocks; a
+    // no-op without PDL), their activations after it.  The ring's entries of
+    // absent batches are zeroed once; copies never touch them.
+    const unsigned char *asrc0[kGemvDepth];
+#pragma unroll
+    for (int d = 0; d < kGemvDepth; ++d) {
+        asrc0[d] = issue_trellis(d);
+        cp_async_commit();
+    }
 #pragma unroll
     for (int d = 0; d < kGemvDepth; ++d)
-        issue(d);
+#pragma unroll
+        for (int o = lane * 16; o < MG * kGemvActBlock; o += 512)
+            *reinterpret_cast<uint4 *>(ring + d * SB + o) = make_uint4(0u, 0u, 0u, 0u);
+    __syncwarp();
+    grid_dep_wait();
+    grid_dep_launch();  // a dependent launch still waits for this grid to complete
+#pragma unroll
+    for (int d = 0; d < kGemvDepth; ++d)
+        if (asrc0[d])
+            copy_acts(d, asrc0[d]);
+    cp_async_commit();
+    cp_async_wait<0>();
     __syncwarp();
 
     const Codebook cb = p.cb;
+    const GemvMults mu = p.mu;
     float acc[MG][8][4];
 #pragma unroll
     for (int a = 0; a < MG; ++a)
@@ -433,16 +526,24 @@ __global__ void __launch_bounds__(kGemvThreads, MG == 1 ? 2 : 1) gemv_kernel(con
             for (int e = 0; e < 4; ++e)
                 acc[a][j][e] = 0.f;
 
-    // the CTA's range as global column blocks [g0, g1]
-    int l0 = 0, c0 = 0, r0 = 0, l1 = 0, c1 = 0, r1 = 0;
-    gemv_locate<MULTI>(p, u0, l0, c0, r0);
-    l1 = l0;
-    gemv_locate<MULTI>(p, u1 - 1, l1, c1, r1);
+    // consumed unit of this warp: cu at (layer cl, column block ccb, tile row
+    // ctr) -- the group's column block cg
+    int64_t cu = u0 + warp;
+    int cl = lb, ccb = 0, ctr = 0;
+    gemv_locate(p, le, cu < u1 ? cu : u0, cl, ccb, ctr);
+    int ctr_lim = p.L[cl].tr_count, cncb = p.L[cl].n >> 7;
+    int cg = p.L[cl].cb_begin + ccb;
+
+    // the CTA's range as the group's column blocks [g0, g1]
+    int l0 = lb, c0 = 0, r0 = 0, c1 = 0, r1 = 0;
+    gemv_locate(p, le, u0, l0, c0, r0);
+    int l1 = l0;
+    gemv_locate(p, le, u1 - 1, l1, c1, r1);
     const int g0 = p.L[l0].cb_begin + c0, g1 = p.L[l1].cb_begin + c1;
     int sl = l0;  // layer of the current segment's column block
     int st = 0;
     for (int gk = g0; gk <= g1; ++gk) {
-        while (MULTI && sl + 1 < p.count && gk >= p.L[sl + 1].cb_begin)
+        while (sl + 1 < le && gk >= p.L[sl + 1].cb_begin)
             ++sl;
         const GemvLayer &SL = p.L[sl];
         const int TR = SL.tr_count;
@@ -450,25 +551,17 @@ __global__ void __launch_bounds__(kGemvThreads, MG == 1 ? 2 : 1) gemv_kernel(con
         while (cu < u1 && cg == gk) {
             cp_async_wait<kGemvDepth - 1>();
             __syncwarp();
-            if (st == 0)
-                mac_stage<K, MG, 0>(lp, cb, acc);
-            else if (st == 1)
-                mac_stage<K, MG, 1>(lp, cb, acc);
-            else
-                mac_stage<K, MG, 2>(lp, cb, acc);
+            mac_unit_at<K, MG, 0>(st, lp, cb, mu, acc);
             __syncwarp();  // every lane is done with the stage before it is refilled
             issue(st);
             st = st + 1 == kGemvDepth ? 0 : st + 1;
             cu += kGemvWarps;
-            // the consumed unit's column block: units advance by 8 <= TR tile rows
             ctr += kGemvWarps;
-            if (ctr >= ctr_lim) {
+            if (ctr >= ctr_lim) {  // 8 <= every TR: at most one column block ahead
                 ctr -= ctr_lim;
                 if (++ccb == cncb) {
                     ccb = 0;
-                    if (MULTI)
-                        ++cl;
-                    if (MULTI && cu < u1) {
+                    if (++cl < le) {
                         ctr_lim = p.L[cl].tr_count;
                         cncb = p.L[cl].n >> 7;
                     }
@@ -480,23 +573,29 @@ __global__ void __launch_bounds__(kGemvThreads, MG == 1 ? 2 : 1) gemv_kernel(con
         const int64_t seg_begin = blk_begin > u0 ? blk_begin : u0;
         const int64_t seg_end = blk_end < u1 ? blk_end : u1;
 
-    // ------------------------------------------- segment end: reduce ---
-        // accumulator (mg, j, e): A row i = g (+8 for e >= 2) -> batch 8mg + i/2,
-        // column parity i&1; n-slot 2t (+1 for odd e) -> tile of the block;
-        // column = 16 * slot + 2j + parity.
+        // ------------------------------------------- segment end: reduce ---
+        // accumulator (mg, j, e): A row g + 8 (e >> 1) -> block column 16g + 2j
+        // + (e >> 1); B column 2t + (e & 1) -> batch 8mg + 2t + (e & 1)
+#pragma unroll
+        for (int mg = 0; mg < MG; ++mg)
+#pragma unroll
+            for (int pb = 0; pb < 2; ++pb) {
+                const int b = 8 * mg + 2 * t + pb;
+                if (b < m) {
+                    float4 *dst = reinterpret_cast<float4 *>(red + (warp * m + b) * 128 + 16 * g);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        dst[q] = make_float4(acc[mg][2 * q][pb], acc[mg][2 * q][2 + pb], acc[mg][2 * q + 1][pb],
+                                             acc[mg][2 * q + 1][2 + pb]);
+                }
+            }
 #pragma unroll
         for (int mg = 0; mg < MG; ++mg)
 #pragma unroll
             for (int j = 0; j < 8; ++j)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int i = g + ((e >> 1) << 3);
-                    const int b = 8 * mg + (i >> 1);
-                    const int col = 16 * (2 * t + (e & 1)) + 2 * j + (i & 1);
-                    if (b < m)
-                        red[(warp * m + b) * 128 + col] = acc[mg][j][e];
+                for (int e = 0; e < 4; ++e)
                     acc[mg][j][e] = 0.f;
-                }
         __syncthreads();
         const int tid = threadIdx.x;
         for (int e = tid; e < m * 128; e += kGemvThreads) {
@@ -511,10 +610,10 @@ __global__ void __launch_bounds__(kGemvThreads, MG == 1 ? 2 : 1) gemv_kernel(con
         if (whole) {
             finish_block(SL, m, red, cbk, warp, lane);
         } else {
-            const int c_first = owner_cta(blk_begin, U, G);
-            const int c_last = owner_cta(blk_end - 1, U, G);
+            const int c_first = (int)gemv_owner_cta(blk_begin, U, G);
+            const int c_last = (int)gemv_owner_cta(blk_end - 1, U, G);
             const int nseg = c_last - c_first + 1;
-            const int j = (int)blockIdx.x - c_first;
+            const int j = (int)c - c_first;
             float *part = SL.partials + ((int64_t)cbk * SL.max_seg) * m * 128;
             for (int e = tid; e < m * 128; e += kGemvThreads)
                 part[(int64_t)j * m * 128 + e] = red[e];
@@ -551,6 +650,27 @@ __global__ void __launch_bounds__(kGemvThreads, MG == 1 ? 2 : 1) gemv_kernel(con
     cp_async_wait<0>();  // nothing may still be landing in shared memory at exit
 }
 
+// The persistent main kernel: each CTA finds its K group and runs the body
+// compiled for that K.
+template <int MG>
+__global__ void __launch_bounds__(kGemvThreads, MG == 1 ? 2 : 1) gemv_kernel(const GemvParams p)
+{
+    int q = 0;
+    while (q + 1 < p.ngroups && (int)blockIdx.x >= p.grp[q + 1].cta_begin)
+        ++q;
+    const GemvGroup &gp = p.grp[q];
+    switch (gp.K) {
+    case 1: gemv_cta<1, MG>(p, gp); break;
+    case 2: gemv_cta<2, MG>(p, gp); break;
+    case 3: gemv_cta<3, MG>(p, gp); break;
+    case 4: gemv_cta<4, MG>(p, gp); break;
+    case 5: gemv_cta<5, MG>(p, gp); break;
+    case 6: gemv_cta<6, MG>(p, gp); break;
+    case 7: gemv_cta<7, MG>(p, gp); break;
+    default: gemv_cta<8, MG>(p, gp); break;
+    }
+}
+
 // ------------------------------------------------------------- dispatch ---
 
 static int g_num_sms = 0;
@@ -570,85 +690,160 @@ int num_sms()
     return g_num_sms;
 }
 
-static int64_t owner_cta_host(int64_t u, int64_t U, int64_t G)
-{
-    return ((u + 1) * G - 1) / U;
-}
-
-// Plan of one launch over `count` layers (same K, same m): grid, shared
-// memory, and the workspace layout -- [0, 256) status word; the layers'
-// arrival counters (one per column block, consecutive); then per layer its
-// activation records (k * 8 MG * 16) and split partials [n/128][max_seg][m][128].
-struct GemvGroupPlan {
-    int ctas, smem;
-    int64_t units;
+// Plan of one launch over `count` layers (same m): the K groups and their
+// CTAs, shared memory, and the workspace layout -- [0, 256) status word; the
+// layers' arrival counters (one per column block, consecutive); then per
+// layer its activation blocks (k / 16 * MG * 512 bytes) and split partials
+// [n/128][max_seg][m][128].  Workspace offsets are indexed by the layer's
+// place in the call; the group order is `order`.
+struct GemvPlan {
+    int ctas, smem, ngroups;
+    GemvGroup grp[8];
+    int order[kGemvMaxLayers];  // call index of the plan's l-th layer (grouped by K)
     int64_t unit_begin[kGemvMaxLayers];
-    int cb_begin[kGemvMaxLayers], max_seg[kGemvMaxLayers];
-    size_t counters[kGemvMaxLayers], recs[kGemvMaxLayers], partials[kGemvMaxLayers], total;
+    int cb_begin[kGemvMaxLayers], max_seg[kGemvMaxLayers];  // by plan index
+    size_t counters[kGemvMaxLayers], acts[kGemvMaxLayers], partials[kGemvMaxLayers], total;  // by call index
 };
+
+// Relative time of one unit at m = 1 by K (measured on B200 with one launch
+// per K: odd K load their runs in 4-byte pieces, larger K move more bytes);
+// it sets each group's share of the grid.
+static int64_t gemv_unit_cost(int K)
+{
+    static const int64_t cost[9] = {0, 330, 335, 373, 351, 395, 384, 415, 406};
+    return cost[K < 1 ? 1 : (K > 8 ? 8 : K)];
+}
 
 // Grid: every CTA resident at once -- resident CTAs per SM from the register
 // budget (2 for m <= 8, 1 above) and the shared memory (228 KB per SM, 1 KB
-// reserved per CTA) -- but at least two units per warp; max_seg = the most
-// CTAs any column block of the layer is split over.
-static GemvGroupPlan gemv_group_plan(const int64_t *k, const int64_t *n, int count, int64_t m, int K, int sms)
+// reserved per CTA) -- split between the K groups in proportion to their
+// cost, each with at least two units per warp; max_seg = the most CTAs any
+// column block of the layer is split over.
+static GemvPlan gemv_plan(const int64_t *k, const int64_t *n, const int *K, int count, int64_t m, int sms)
 {
-    GemvGroupPlan pl;
-    pl.units = 0;
-    int cb = 0;
-    for (int l = 0; l < count; ++l) {
-        pl.unit_begin[l] = pl.units;
-        pl.cb_begin[l] = cb;
-        pl.units += (k[l] / 16) * (n[l] / 128);
-        cb += (int)(n[l] / 128);
+    GemvPlan pl;
+    const int MG = gemv_mg(m);
+    pl.ngroups = 0;
+    int np = 0, max_sb = 0;
+    for (int kk = 1; kk <= 8; ++kk) {
+        GemvGroup gr;
+        gr.K = kk;
+        gr.l_begin = np;
+        gr.units = 0;
+        int cbn = 0;
+        for (int l = 0; l < count; ++l) {
+            if (K[l] != kk)
+                continue;
+            pl.order[np] = l;
+            pl.unit_begin[np] = gr.units;
+            pl.cb_begin[np] = cbn;
+            gr.units += (k[l] / 16) * (n[l] / 128);
+            cbn += (int)(n[l] / 128);
+            ++np;
+        }
+        gr.l_end = np;
+        if (gr.l_end > gr.l_begin) {
+            pl.grp[pl.ngroups++] = gr;
+            const int sb = gemv_stage_bytes(kk, MG);
+            max_sb = sb > max_sb ? sb : max_sb;
+        }
     }
-    pl.smem = 128 + kGemvWarps * kGemvDepth * gemv_stage_bytes(K, gemv_mg(m)) + kGemvWarps * (int)m * 128 * 4;
+    pl.smem = 128 + kGemvWarps * (int)m * 128 * 4 + kGemvWarps * kGemvDepth * max_sb;
     int64_t occ = m <= 8 ? 2 : 1;
     const int64_t occ_smem = (228 * 1024) / (pl.smem + 1024);
     if (occ_smem < occ)
         occ = occ_smem > 0 ? occ_smem : 1;
-    int64_t G = occ * (int64_t)sms;
-    const int64_t gmax = pl.units / (2 * kGemvWarps);  // at least 2 units per warp
-    if (G > gmax)
-        G = gmax > 0 ? gmax : 1;
+    const int64_t G = occ * (int64_t)sms;
+
+    // CTAs per group: proportional to cost (largest remainder), at least 1,
+    // at most units / 16 (two units per warp)
+    int64_t cost_sum = 0;
+    for (int q = 0; q < pl.ngroups; ++q)
+        cost_sum += pl.grp[q].units * gemv_unit_cost(pl.grp[q].K);
+    int64_t given = 0;
+    int64_t rem[8];
+    for (int q = 0; q < pl.ngroups; ++q) {
+        const int64_t num = G * pl.grp[q].units * gemv_unit_cost(pl.grp[q].K);
+        int64_t gq = num / cost_sum;
+        rem[q] = num - gq * cost_sum;
+        const int64_t cap = pl.grp[q].units / (2 * kGemvWarps) > 0 ? pl.grp[q].units / (2 * kGemvWarps) : 1;
+        gq = gq < 1 ? 1 : (gq > cap ? cap : gq);
+        pl.grp[q].ctas = (int)gq;
+        given += gq;
+    }
+    while (given < G) {  // hand out what rounding left, largest remainder first
+        int best = -1;
+        for (int q = 0; q < pl.ngroups; ++q) {
+            const int64_t cap = pl.grp[q].units / (2 * kGemvWarps);
+            if (pl.grp[q].ctas < cap && (best < 0 || rem[q] > rem[best]))
+                best = q;
+        }
+        if (best < 0)
+            break;
+        ++pl.grp[best].ctas;
+        rem[best] = -1;
+        ++given;
+        bool any = false;
+        for (int q = 0; q < pl.ngroups; ++q)
+            any = any || rem[q] >= 0;
+        if (!any)
+            for (int q = 0; q < pl.ngroups; ++q)
+                rem[q] = 0;
+    }
     if (count == 1) {
         // A whole number of CTAs per column block aligns the CTA ranges with
         // the column blocks, so no CTA straddles two (one segment end instead
         // of two, each about as costly as 8 units).  Take it when the busiest
         // SM's modelled work (units + 8 per segment end) is lower.
+        GemvGroup &gr = pl.grp[0];
+        const int64_t Gq = gr.ctas;
         const int64_t ncb = n[0] / 128;
-        const int64_t s_blk = G / ncb;
-        if (s_blk >= 1 && s_blk * ncb != G) {
-            auto cost = [&](int64_t g, int64_t segs) {
-                const int64_t per_sm = (g + sms - 1) / sms;
-                return (pl.units + g - 1) / g * per_sm + 8 * segs * per_sm;
+        const int64_t s_blk = Gq / ncb;
+        if (s_blk >= 1 && s_blk * ncb != Gq) {
+            auto cost = [&](int64_t gg, int64_t segs) {
+                const int64_t per_sm = (gg + sms - 1) / sms;
+                return (gr.units + gg - 1) / gg * per_sm + 8 * segs * per_sm;
             };
-            if (cost(s_blk * ncb, 1) < cost(G, 2))
-                G = s_blk * ncb;
+            if (cost(s_blk * ncb, 1) < cost(Gq, 2))
+                gr.ctas = (int)(s_blk * ncb);
         }
     }
-    pl.ctas = (int)G;
+    int cta = 0;
+    for (int q = 0; q < pl.ngroups; ++q) {
+        pl.grp[q].cta_begin = cta;
+        cta += pl.grp[q].ctas;
+    }
+    pl.ctas = cta;
+
     size_t off = 256;
     for (int l = 0; l < count; ++l) {
         pl.counters[l] = off;
         off += (size_t)(n[l] / 128) * 4;
     }
     off = (off + 255) / 256 * 256;
-    for (int l = 0; l < count; ++l) {
-        const int64_t TR = k[l] / 16, ncb = n[l] / 128;
-        int64_t max_seg = 1;
-        for (int64_t c = 0; c < ncb; ++c) {
-            const int64_t b0 = pl.unit_begin[l] + c * TR;
-            const int64_t s = owner_cta_host(b0 + TR - 1, pl.units, G) - owner_cta_host(b0, pl.units, G) + 1;
-            max_seg = s > max_seg ? s : max_seg;
+    for (int q = 0; q < pl.ngroups; ++q) {
+        const GemvGroup &gr = pl.grp[q];
+        for (int i = gr.l_begin; i < gr.l_end; ++i) {
+            const int l = pl.order[i];
+            const int64_t TR = k[l] / 16, ncb = n[l] / 128;
+            int64_t max_seg = 1;
+            for (int64_t c = 0; c < ncb; ++c) {
+                const int64_t b0 = pl.unit_begin[i] + c * TR;
+                const int64_t sg =
+                    gemv_owner_cta(b0 + TR - 1, gr.units, gr.ctas) - gemv_owner_cta(b0, gr.units, gr.ctas) + 1;
+                max_seg = sg > max_seg ? sg : max_seg;
+            }
+            pl.max_seg[i] = (int)max_seg;
         }
-        pl.max_seg[l] = (int)max_seg;
-        pl.recs[l] = off;
-        off += ((size_t)k[l] * rec_slots_for(gemv_mg(m)) * 16 + 255) / 256 * 256;
     }
     for (int l = 0; l < count; ++l) {
+        pl.acts[l] = off;
+        off += ((size_t)(k[l] / 16) * MG * kGemvActBlock + 255) / 256 * 256;
+    }
+    for (int i = 0; i < count; ++i) {
+        const int l = pl.order[i];
         pl.partials[l] = off;
-        off += ((size_t)(n[l] / 128) * (size_t)pl.max_seg[l] * (size_t)m * 128 * 4 + 255) / 256 * 256;
+        off += ((size_t)(n[l] / 128) * (size_t)pl.max_seg[i] * (size_t)m * 128 * 4 + 255) / 256 * 256;
     }
     pl.total = off;
     return pl;
@@ -658,42 +853,15 @@ size_t gemv_workspace_bytes(int64_t m, int64_t k, int64_t n, int sms)
 {
     size_t most = 0;
     for (int K = 1; K <= 8; ++K) {
-        const size_t b = gemv_group_plan(&k, &n, 1, m, K, sms).total;
+        const size_t b = gemv_plan(&k, &n, &K, 1, m, sms).total;
         most = b > most ? b : most;
     }
     return most;
 }
 
-template <int K, int MG>
-static exl3_status launch_gemv_t(const GemvParams &p, int smem, cudaStream_t stream)
-{
-    auto kern = p.count > 1 ? gemv_kernel<K, MG, true> : gemv_kernel<K, MG, false>;
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-        return EXL3_ERR_CUDA;
-    if (launch_kernel(kern, dim3((unsigned)p.ctas), dim3(kGemvThreads), (size_t)smem, stream, p) != cudaSuccess)
-        return EXL3_ERR_CUDA;
-    return launch_status();
-}
-
-template <int MG>
-static exl3_status launch_gemv_k(const GemvParams &p, int K, int smem, cudaStream_t stream)
-{
-    switch (K) {
-    case 1: return launch_gemv_t<1, MG>(p, smem, stream);
-    case 2: return launch_gemv_t<2, MG>(p, smem, stream);
-    case 3: return launch_gemv_t<3, MG>(p, smem, stream);
-    case 4: return launch_gemv_t<4, MG>(p, smem, stream);
-    case 5: return launch_gemv_t<5, MG>(p, smem, stream);
-    case 6: return launch_gemv_t<6, MG>(p, smem, stream);
-    case 7: return launch_gemv_t<7, MG>(p, smem, stream);
-    default: return launch_gemv_t<8, MG>(p, smem, stream);
-    }
-}
-
-// Launches the rotation kernel over `count` (<= kGemvRotMaxLayers) layers:
-// layer l's records go to recs[l].
-static exl3_status launch_rotation(const exl3_linear *const *layers, unsigned char *const *recs, int count,
+// Launches the rotation kernel over `count` (<= kGemvMaxLayers) layers:
+// layer l's activation blocks go to acts[l].
+static exl3_status launch_rotation(const exl3_linear *const *layers, unsigned char *const *acts, int count,
                                    int64_t m, cudaStream_t stream)
 {
     const int sms = num_sms();
@@ -701,14 +869,13 @@ static exl3_status launch_rotation(const exl3_linear *const *layers, unsigned ch
     rp.count = count;
     rp.m = (int)m;
     int64_t jobs = 0;
-    const int quads = rec_quads((int)m, 0) + rec_quads((int)m, 1);
     for (int l = 0; l < count; ++l) {
         rp.L[l].x = (const __half *)layers[l]->x;
         rp.L[l].suh = (const __half *)layers[l]->suh;
-        rp.L[l].recs = recs[l];
+        rp.L[l].acts = acts[l];
         rp.L[l].k = (int)layers[l]->k;
         rp.L[l].job_begin = jobs;
-        jobs += (int64_t)quads * (layers[l]->k / 128);
+        jobs += m * (layers[l]->k / 128);
     }
     rp.jobs = jobs;
     int64_t rgrid = (jobs + 7) / 8;
@@ -721,54 +888,62 @@ static exl3_status launch_rotation(const exl3_linear *const *layers, unsigned ch
     return launch_status();
 }
 
-// The main launch over up to kGemvMaxLayers layers of the same K, with the
-// workspace region `ws` laid out by gemv_group_plan; with `rotate` it first
-// launches the rotation for them (else their records are already in place).
-static exl3_status run_gemv_group(const exl3_linear *const *layers, int count, int64_t m, int K,
-                                  unsigned char *ws, size_t ws_bytes, cudaStream_t stream, bool rotate = true)
+// One rotation launch and one main launch over up to kGemvMaxLayers layers,
+// with the workspace region `ws` laid out by gemv_plan.
+static exl3_status run_gemv_launch(const exl3_linear *const *layers, int count, int64_t m, unsigned char *ws,
+                                   size_t ws_bytes, cudaStream_t stream)
 {
     const int sms = num_sms();
     int64_t k[kGemvMaxLayers], n[kGemvMaxLayers];
+    int K[kGemvMaxLayers];
     for (int l = 0; l < count; ++l) {
         k[l] = layers[l]->k;
         n[l] = layers[l]->n;
+        K[l] = layers[l]->K;
     }
-    const GemvGroupPlan pl = gemv_group_plan(k, n, count, m, K, sms);
+    const GemvPlan pl = gemv_plan(k, n, K, count, m, sms);
     if (!ws || !aligned16(ws) || ws_bytes < pl.total)
         return EXL3_ERR_WORKSPACE;
 
-    if (rotate) {
-        unsigned char *recs[kGemvMaxLayers];
-        for (int l = 0; l < count; ++l)
-            recs[l] = ws + pl.recs[l];
-        const exl3_status rs = launch_rotation(layers, recs, count, m, stream);
-        if (rs != EXL3_OK)
-            return rs;
-    }
+    unsigned char *acts[kGemvMaxLayers];
+    for (int l = 0; l < count; ++l)
+        acts[l] = ws + pl.acts[l];
+    const exl3_status rs = launch_rotation(layers, acts, count, m, stream);
+    if (rs != EXL3_OK)
+        return rs;
 
     GemvParams p;
-    p.count = count;
     p.m = (int)m;
-    p.ctas = pl.ctas;
-    p.units = pl.units;
+    p.ngroups = pl.ngroups;
+    for (int q = 0; q < pl.ngroups; ++q)
+        p.grp[q] = pl.grp[q];
     p.cb = codebook_constants();
-    for (int l = 0; l < count; ++l) {
-        GemvLayer &L = p.L[l];
+    for (int i = 0; i < 8; ++i)
+        p.mu.pow2[i] = 1u << i;
+    p.mu.hi16 = 1u << 16;
+    for (int i = 0; i < count; ++i) {
+        const int l = pl.order[i];
+        GemvLayer &L = p.L[i];
         L.trellis = reinterpret_cast<const unsigned char *>(layers[l]->trellis);
         L.svh = (const __half *)layers[l]->svh;
         L.y = (__half *)layers[l]->y;
-        L.recs = ws + pl.recs[l];
+        L.acts = ws + pl.acts[l];
         L.partials = reinterpret_cast<float *>(ws + pl.partials[l]);
         L.counters = reinterpret_cast<uint32_t *>(ws + pl.counters[l]);
-        L.unit_begin = pl.unit_begin[l];
+        L.unit_begin = pl.unit_begin[i];
         L.n = (int)n[l];
         L.tr_count = (int)(k[l] / 16);
-        L.cb_begin = pl.cb_begin[l];
-        L.max_seg = pl.max_seg[l];
+        L.max_seg = pl.max_seg[i];
+        L.cb_begin = pl.cb_begin[i];
     }
-    if (m <= 8)
-        return launch_gemv_k<1>(p, K, pl.smem, stream);
-    return launch_gemv_k<2>(p, K, pl.smem, stream);
+    auto kern = m <= 8 ? gemv_kernel<1> : gemv_kernel<2>;
+    if (pl.smem > 48 * 1024 &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem) != cudaSuccess)
+        return EXL3_ERR_CUDA;
+    if (launch_kernel(kern, dim3((unsigned)pl.ctas), dim3(kGemvThreads), (size_t)pl.smem, stream, p) !=
+        cudaSuccess)
+        return EXL3_ERR_CUDA;
+    return launch_status();
 }
 
 exl3_status run_gemv(const void *x, const uint16_t *trellis, const void *suh, const void *svh,
@@ -785,37 +960,32 @@ exl3_status run_gemv(const void *x, const uint16_t *trellis, const void *suh, co
     d.n = n;
     d.K = K;
     const exl3_linear *one = &d;
-    return run_gemv_group(&one, 1, m, K, (unsigned char *)workspace, workspace_bytes, stream);
+    return run_gemv_launch(&one, 1, m, (unsigned char *)workspace, workspace_bytes, stream);
 }
 
-// The layers of a multi call, grouped by K (in call order) into launches of
-// at most kGemvMaxLayers; calls f(group, count, K, workspace offset, bytes).
+// The layers of a multi call in launches of at most kGemvMaxLayers, in call
+// order; calls f(layers, count, workspace offset, bytes) per launch.
 template <typename F>
-static exl3_status for_each_gemv_group(const exl3_linear *layers, int count, int64_t m, F &&f)
+static exl3_status for_each_gemv_launch(const exl3_linear *layers, int count, int64_t m, F &&f)
 {
     const int sms = num_sms();
     size_t off = 0;
-    for (int K = 1; K <= 8; ++K) {
+    for (int first = 0; first < count; first += kGemvMaxLayers) {
+        const int cnt = count - first < kGemvMaxLayers ? count - first : kGemvMaxLayers;
         const exl3_linear *grp[kGemvMaxLayers];
-        int cnt = 0;
-        for (int i = 0; i <= count; ++i) {
-            const bool flush = (i == count && cnt > 0) || cnt == kGemvMaxLayers;
-            if (flush) {
-                int64_t k[kGemvMaxLayers], n[kGemvMaxLayers];
-                for (int l = 0; l < cnt; ++l) {
-                    k[l] = grp[l]->k;
-                    n[l] = grp[l]->n;
-                }
-                const size_t bytes = gemv_group_plan(k, n, cnt, m, K, sms).total;
-                const exl3_status st = f(grp, cnt, K, off, bytes);
-                if (st != EXL3_OK)
-                    return st;
-                off += (bytes + 255) / 256 * 256;
-                cnt = 0;
-            }
-            if (i < count && layers[i].K == K)
-                grp[cnt++] = &layers[i];
+        int64_t k[kGemvMaxLayers], n[kGemvMaxLayers];
+        int K[kGemvMaxLayers];
+        for (int l = 0; l < cnt; ++l) {
+            grp[l] = &layers[first + l];
+            k[l] = grp[l]->k;
+            n[l] = grp[l]->n;
+            K[l] = grp[l]->K;
         }
+        const size_t bytes = gemv_plan(k, n, K, cnt, m, sms).total;
+        const exl3_status st = f(grp, cnt, off, bytes);
+        if (st != EXL3_OK)
+            return st;
+        off += (bytes + 255) / 256 * 256;
     }
     return EXL3_OK;
 }
@@ -863,7 +1033,7 @@ extern "C" size_t exl3_gemv_multi_workspace_size(const exl3_linear *layers, int 
     if (check_multi(layers, count, m) != EXL3_OK)
         return 0;
     size_t total = 0;
-    for_each_gemv_group(layers, count, m, [&](const exl3_linear *const *, int, int, size_t off, size_t bytes) {
+    for_each_gemv_launch(layers, count, m, [&](const exl3_linear *const *, int, size_t off, size_t bytes) {
         total = off + (bytes + 255) / 256 * 256;
         return EXL3_OK;
     });
@@ -880,41 +1050,10 @@ extern "C" exl3_status exl3_gemv_multi(const exl3_linear *layers, int count, int
     if (!workspace || !aligned16(workspace) || workspace_bytes < exl3_gemv_multi_workspace_size(layers, count, m))
         return EXL3_ERR_WORKSPACE;
     unsigned char *ws = (unsigned char *)workspace;
-    cudaStream_t s = (cudaStream_t)stream;
-    // every layer's rotation first, in launches of up to kGemvRotMaxLayers
-    // layers, then one main launch per group reading its records
-    const int sms = num_sms();
-    const exl3_linear *rl[kGemvRotMaxLayers];
-    unsigned char *rr[kGemvRotMaxLayers];
-    int nr = 0;
-    exl3_status st2 = for_each_gemv_group(
-        layers, count, m, [&](const exl3_linear *const *grp, int cnt, int K, size_t off, size_t) {
-            int64_t k[kGemvMaxLayers], n[kGemvMaxLayers];
-            for (int l = 0; l < cnt; ++l) {
-                k[l] = grp[l]->k;
-                n[l] = grp[l]->n;
-            }
-            const GemvGroupPlan pl = gemv_group_plan(k, n, cnt, m, K, sms);
-            for (int l = 0; l < cnt; ++l) {
-                rl[nr] = grp[l];
-                rr[nr] = ws + off + pl.recs[l];
-                if (++nr == kGemvRotMaxLayers) {
-                    const exl3_status rs = launch_rotation(rl, rr, nr, m, s);
-                    if (rs != EXL3_OK)
-                        return rs;
-                    nr = 0;
-                }
-            }
-            return EXL3_OK;
-        });
-    if (st2 == EXL3_OK && nr > 0)
-        st2 = launch_rotation(rl, rr, nr, m, s);
-    if (st2 != EXL3_OK)
-        return st2;
-    return for_each_gemv_group(layers, count, m,
-                               [&](const exl3_linear *const *grp, int cnt, int K, size_t off, size_t bytes) {
-                                   return run_gemv_group(grp, cnt, m, K, ws + off, bytes, s, false);
-                               });
+    return for_each_gemv_launch(layers, count, m,
+                                [&](const exl3_linear *const *grp, int cnt, size_t off, size_t bytes) {
+                                    return run_gemv_launch(grp, cnt, m, ws + off, bytes, (cudaStream_t)stream);
+                                });
 }
 
 // ------------------------------------------------ no-allocation variant ---
