@@ -58,7 +58,7 @@ constexpr int kGemvThreads = 32 * kGemvWarps;
 // (tr * MG + mg) * 512.  Only batches < m are written and copied; the ring's
 // entries of absent batches are zero (they feed only B columns whose
 // accumulators are never stored).
-__host__ __device__ constexpr int kGemvActBlock = 512;
+constexpr int kGemvActBlock = 512;
 
 __host__ __device__ inline int gemv_mg(int64_t m)
 {
@@ -432,23 +432,28 @@ __device__ __forceinline__ void gemv_cta(const GemvParams &p, const GemvGroup &g
     for (int mg = 0; mg < MG; ++mg)
         act_live[mg] = 8 * mg + ((lane >> 1) & 7) < m;
 
-    // issue iterator (runs kGemvDepth units ahead of consumption): unit iu at
-    // (layer il, column block icb, tile row itr), advancing by 8 units
-    int64_t iu = u0 + warp;
+    // this warp's units: u0 + warp + 8i, i < nunits
+    const int nunits = u0 + warp < u1 ? (int)((u1 - u0 - warp + 7) >> 3) : 0;
+
+    // issue iterator (runs kGemvDepth units ahead of consumption): the next
+    // unit to copy is at (layer il, column block icb, tile row itr); `rem`
+    // units are left to copy
+    int rem = nunits;
     int il = lb, icb = 0, itr = 0;
-    gemv_locate(p, le, iu < u1 ? iu : u0, il, icb, itr);
+    gemv_locate(p, le, rem ? u0 + warp : u0, il, icb, itr);
     int itr_lim = 0, incb = 0;
-    int64_t tile_row_bytes = 0;
+    int64_t tile_rows8 = 0;  // 8 tile rows of the layer's matrix, in bytes
     const unsigned char *isrc = nullptr, *iasrc = nullptr;
     auto enter_block = [&]() {
         const GemvLayer &L = p.L[il];
         itr_lim = L.tr_count;
         incb = L.n >> 7;
-        tile_row_bytes = (int64_t)(L.n >> 4) * 32 * K;
+        const int64_t tile_row_bytes = (int64_t)(L.n >> 4) * 32 * K;
+        tile_rows8 = kGemvWarps * tile_row_bytes;
         isrc = L.trellis + itr * tile_row_bytes + (int64_t)icb * 256 * K + lane * 16;
         iasrc = L.acts + (int64_t)itr * MG * kGemvActBlock + lane * 16;
     };
-    if (iu < u1)
+    if (rem)
         enter_block();
     auto copy_acts = [&](int stage, const unsigned char *src) {
 #pragma unroll
@@ -456,36 +461,33 @@ __device__ __forceinline__ void gemv_cta(const GemvParams &p, const GemvGroup &g
             if (act_live[mg])
                 cp_async16(ring + stage * SB + mg * kGemvActBlock + lane * 16, src + mg * kGemvActBlock);
     };
-    // copies the trellis of the issue iterator's unit into `stage`, returns
-    // the unit's activation source (null past the range) and advances
+    // copies the trellis of the issue iterator's unit into `stage` (rem > 0),
+    // returns the unit's activation source and advances by 8 units
     auto issue_trellis = [&](int stage) -> const unsigned char * {
-        if (iu >= u1)
-            return nullptr;
         const unsigned char *asrc = iasrc;
         const int so = stage * SB;
 #pragma unroll
         for (int r = 0; r < kTrChunks; ++r)
             if (r < kTrChunks - 1 || last_chunk)
                 cp_async16(tdst[r] + so, isrc + 512 * r);
-        iu += kGemvWarps;
-        itr += kGemvWarps;
-        isrc += kGemvWarps * tile_row_bytes;
+        --rem;
+        isrc += tile_rows8;
         iasrc += kGemvWarps * MG * kGemvActBlock;
+        itr += kGemvWarps;
         if (itr >= itr_lim) {  // next column block, perhaps of the next layer (8 <= every TR)
             itr -= itr_lim;
             if (++icb == incb) {
                 icb = 0;
                 ++il;
             }
-            if (iu < u1)
+            if (rem)
                 enter_block();
         }
         return asrc;
     };
     auto issue = [&](int stage) {
-        const unsigned char *asrc = issue_trellis(stage);
-        if (asrc)
-            copy_acts(stage, asrc);
+        if (rem > 0)
+            copy_acts(stage, issue_trellis(stage));
         cp_async_commit();
     };
 
@@ -496,7 +498,7 @@ __device__ __forceinline__ void gemv_cta(const GemvParams &p, const GemvGroup &g
     const unsigned char *asrc0[kGemvDepth];
 #pragma unroll
     for (int d = 0; d < kGemvDepth; ++d) {
-        asrc0[d] = issue_trellis(d);
+        asrc0[d] = rem > 0 ? issue_trellis(d) : nullptr;
         cp_async_commit();
     }
 #pragma unroll
@@ -526,14 +528,6 @@ __device__ __forceinline__ void gemv_cta(const GemvParams &p, const GemvGroup &g
             for (int e = 0; e < 4; ++e)
                 acc[a][j][e] = 0.f;
 
-    // consumed unit of this warp: cu at (layer cl, column block ccb, tile row
-    // ctr) -- the group's column block cg
-    int64_t cu = u0 + warp;
-    int cl = lb, ccb = 0, ctr = 0;
-    gemv_locate(p, le, cu < u1 ? cu : u0, cl, ccb, ctr);
-    int ctr_lim = p.L[cl].tr_count, cncb = p.L[cl].n >> 7;
-    int cg = p.L[cl].cb_begin + ccb;
-
     // the CTA's range as the group's column blocks [g0, g1]
     int l0 = lb, c0 = 0, r0 = 0, c1 = 0, r1 = 0;
     gemv_locate(p, le, u0, l0, c0, r0);
@@ -542,36 +536,27 @@ __device__ __forceinline__ void gemv_cta(const GemvParams &p, const GemvGroup &g
     const int g0 = p.L[l0].cb_begin + c0, g1 = p.L[l1].cb_begin + c1;
     int sl = l0;  // layer of the current segment's column block
     int st = 0;
+    int ci = 0;  // units consumed
     for (int gk = g0; gk <= g1; ++gk) {
         while (sl + 1 < le && gk >= p.L[sl + 1].cb_begin)
             ++sl;
         const GemvLayer &SL = p.L[sl];
         const int TR = SL.tr_count;
         const int cbk = gk - SL.cb_begin;  // column block within the layer
-        while (cu < u1 && cg == gk) {
+        const int64_t blk_begin = SL.unit_begin + (int64_t)cbk * TR, blk_end = blk_begin + TR;
+        const int64_t seg_begin = blk_begin > u0 ? blk_begin : u0;
+        const int64_t seg_end = blk_end < u1 ? blk_end : u1;
+        // this warp's units below seg_end: ceil((seg_end - u0 - warp) / 8)
+        const int rel_end = (int)(seg_end - u0) - warp;
+        const int upto = rel_end > 0 ? (rel_end + kGemvWarps - 1) / kGemvWarps : 0;
+        for (; ci < upto; ++ci) {
             cp_async_wait<kGemvDepth - 1>();
             __syncwarp();
             mac_unit_at<K, MG, 0>(st, lp, cb, mu, acc);
             __syncwarp();  // every lane is done with the stage before it is refilled
             issue(st);
             st = st + 1 == kGemvDepth ? 0 : st + 1;
-            cu += kGemvWarps;
-            ctr += kGemvWarps;
-            if (ctr >= ctr_lim) {  // 8 <= every TR: at most one column block ahead
-                ctr -= ctr_lim;
-                if (++ccb == cncb) {
-                    ccb = 0;
-                    if (++cl < le) {
-                        ctr_lim = p.L[cl].tr_count;
-                        cncb = p.L[cl].n >> 7;
-                    }
-                }
-                cg = cu < u1 ? p.L[cl].cb_begin + ccb : cg + 1;
-            }
         }
-        const int64_t blk_begin = SL.unit_begin + (int64_t)cbk * TR, blk_end = blk_begin + TR;
-        const int64_t seg_begin = blk_begin > u0 ? blk_begin : u0;
-        const int64_t seg_end = blk_end < u1 ? blk_end : u1;
 
         // ------------------------------------------- segment end: reduce ---
         // accumulator (mg, j, e): A row g + 8 (e >> 1) -> block column 16g + 2j
