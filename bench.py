@@ -393,7 +393,7 @@ def run_ours(args, rank, world, local_rank):
         w_clk_sm = weights / (ms * 1e-3) / (sms * sm_hz * 1e6)
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
-                "traffic_unit": "bytes per step (ncu dram read + write, all 40 launches of a step)",
+                "traffic_unit": "bytes per step (ncu dram read + write of the step's rotation and main launch)",
                 "algorithmic_bytes_per_step": step_bytes,
                 "kernel": "exl3_gemv_multi over the 20 layers: one gemv_rotate_kernel + one persistent "
                           "gemv_kernel whose CTAs are split into K groups (%d launch pair(s)); duration = timed "
