@@ -48,6 +48,13 @@ def _load():
         lib.oracle_linear.argtypes = [u16p, u16p, u16p, u16p, i64, i64, i64, ctypes.c_int,
                                       i64, i64, f64p, ctypes.c_int]
         lib.oracle_linear.restype = None
+        f32p = ctypes.POINTER(ctypes.c_float)
+        u8p = ctypes.POINTER(ctypes.c_uint8)
+        lib.oracle_encode_seq.argtypes = [f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, f32p, u8p, f32p,
+                                          ctypes.POINTER(ctypes.c_int)]
+        lib.oracle_encode_seq.restype = ctypes.c_int
+        lib.oracle_encode.argtypes = [f32p, i64, i64, ctypes.c_int, u16p, f32p, ctypes.c_int]
+        lib.oracle_encode.restype = ctypes.c_int
         lib.oracle_threads_available.argtypes = []
         lib.oracle_threads_available.restype = ctypes.c_int
         _lib = lib
@@ -147,9 +154,41 @@ def linear(x, trellis, suh, svh, K, col_blocks=None, threads=1):
     return y
 
 
+def encode_seq(target, L, K, cb):
+    """Tail-biting Viterbi encoding of one sequence on an L-bit trellis with K
+    bits per weight and state values cb (2^L floats).  Returns (chunks, cost,
+    overlap): each weight's K new bits, the fp32 squared-error sum of the
+    closed path, and the overlap (low L-K bits of the last state)."""
+    t = np.ascontiguousarray(target, dtype=np.float32)
+    c = np.ascontiguousarray(cb, dtype=np.float32)
+    assert c.size == 1 << L and 2 * K <= L
+    chunks = np.empty(t.size, dtype=np.uint8)
+    cost = ctypes.c_float()
+    o = ctypes.c_int()
+    rc = _load().oracle_encode_seq(_ptr(t, ctypes.c_float), int(t.size), int(L), int(K), _ptr(c, ctypes.c_float),
+                                   _ptr(chunks, ctypes.c_uint8), ctypes.byref(cost), ctypes.byref(o))
+    assert rc == 0
+    return chunks, float(cost.value), int(o.value)
+
+
+def encode(w, K, threads=1):
+    """Encodes a k x n float32 matrix into the trellis layout [k/16][n/16][16K]
+    (uint16).  Returns (trellis, cost): cost[tk, tn] is the tile's fp32
+    squared-error sum."""
+    a = np.ascontiguousarray(w, dtype=np.float32)
+    k, n = a.shape
+    assert k % 16 == 0 and n % 16 == 0
+    trellis = np.empty((k // 16, n // 16, 16 * K), dtype=np.uint16)
+    cost = np.empty((k // 16, n // 16), dtype=np.float32)
+    rc = _load().oracle_encode(_ptr(a, ctypes.c_float), k, n, int(K), _ptr(trellis, ctypes.c_uint16),
+                               _ptr(cost, ctypes.c_float), int(threads))
+    assert rc == 0
+    return trellis, cost
+
+
 def threads_available():
     return int(_load().oracle_threads_available())
 
 
 __all__ = ["half_to_double", "double_to_half", "codebook_table", "codebook", "state", "states",
-           "decode_tiles", "hadamard", "linear", "threads_available"]
+           "decode_tiles", "hadamard", "linear", "encode_seq", "encode", "threads_available"]

@@ -22,6 +22,10 @@
  *     normalised (EXL3 GEMM kernel article, section "GEMM内核": the kernel
  *     rotates the input A with a 128-point Hadamard before the matmul).
  *   - the linear layer y = x . W_hat with both rotations, in fp64.
+ *   - the tail-biting trellis encoder: for each 16x16 tile, the Viterbi
+ *     search for the bit string whose decoded weights are closest (squared
+ *     error) to the tile's target values (EXL3 GEMM kernel article, section
+ *     "Viterbi编码内核剖析"; readings at oracle_encode_seq).
  *
  * Readings of points the pages leave open (the pages give no bit order, tile
  * layout or normalisation):
@@ -156,6 +160,141 @@ void oracle_decode_tiles(const uint16_t *trellis, int64_t k, int64_t n, int K, u
                 w[(tk * 16 + r) * n + tn * 16 + c] = oracle_codebook(oracle_state(tile, K, i));
             }
         }
+}
+
+/* ------------------------------------------------------------- encoder -- */
+
+/* Tail-biting Viterbi encoding of one sequence (EXL3 GEMM kernel article,
+ * section "Viterbi编码内核剖析": a 16x16 block of weights is encoded by a
+ * Viterbi forward pass over the trellis that keeps the accumulated cost of
+ * every path and takes the cheapest; the tail-biting boundary is closed by
+ * enumerating start states, so that the codeword's head and tail agree).
+ *
+ * Generic in the trellis size so that tests can compare it with exhaustive
+ * search on a small trellis: T weights, L-bit states (16 for EXL3), K bits
+ * per weight (2K <= L), and the value of every state in `cb` (2^L floats;
+ * for EXL3 the codebook).  The state of weight i is s_i = ((s_{i-1} << K) |
+ * c_i) mod 2^L with c_i the weight's K new bits, and the code is tail-biting:
+ * s_{-1} = s_{T-1}.
+ *
+ * Readings of what the pages leave open:
+ *   - the cost of weight i in state s is (target_i - cb[s])^2, formed in fp32
+ *     as fmaf(d, d, path cost) with d = target_i - cb[s] rounded to fp32 (the
+ *     precision in which the GPU kernel takes the same decisions);
+ *   - M_i[m] is the cheapest cost of a path through weight i whose state has
+ *     low L-K bits m, i.e. the states that can precede a state whose high
+ *     L-K bits are m: M_i[m] = min over h of fmaf(d, d, M_{i-1}[s >> K]) with
+ *     s = (h << (L-K)) | m, the smallest h winning ties; h is recorded;
+ *   - pass 1 enumerates every start state (M_{-1} = 0 everywhere).  The
+ *     cheapest end, o = argmin_m M_{T-1}[m] (smallest m on ties), fixes the
+ *     overlap: the low L-K bits of the last state, which a tail-biting code
+ *     repeats as the high L-K bits of the first;
+ *   - pass 2 closes the loop: M_{-1}[x] = 0 for x == o and +inf otherwise, so
+ *     the first state's high bits are o; the path ends in the cheapest state
+ *     with low bits o and is traced back through the recorded choices.
+ * Outputs: chunks[i] = c_i (the low K bits of s_i), the pass-2 path cost
+ * (fp32) and the overlap o.  Returns 0, or -1 if memory runs out. */
+int oracle_encode_seq(const float *target, int T, int L, int K, const float *cb, unsigned char *chunks,
+                      float *cost, int *overlap)
+{
+    const long nm = 1L << (L - K), nh = 1L << K;
+    float *prev = (float *)malloc(sizeof(float) * nm);
+    float *next = (float *)malloc(sizeof(float) * nm);
+    unsigned char *choice = (unsigned char *)malloc((size_t)T * (size_t)nm);
+    if (!prev || !next || !choice) {
+        free(prev);
+        free(next);
+        free(choice);
+        return -1;
+    }
+    int o = 0;
+    for (int pass = 1; pass <= 2; ++pass) {
+        for (long m = 0; m < nm; ++m)
+            prev[m] = (pass == 1 || m == o) ? 0.0f : INFINITY;
+        for (int i = 0; i < T; ++i) {
+            for (long m = 0; m < nm; ++m) {
+                float best = 0.0f;
+                int best_h = 0;
+                for (long h = 0; h < nh; ++h) {
+                    const long s = (h << (L - K)) | m;
+                    const float d = target[i] - cb[s];
+                    const float v = fmaf(d, d, prev[s >> K]);
+                    if (h == 0 || v < best) {
+                        best = v;
+                        best_h = (int)h;
+                    }
+                }
+                next[m] = best;
+                choice[(size_t)i * (size_t)nm + (size_t)m] = (unsigned char)best_h;
+            }
+            float *t = prev;
+            prev = next;
+            next = t;
+        }
+        if (pass == 1) {
+            o = 0;
+            for (long m = 1; m < nm; ++m)
+                if (prev[m] < prev[o])
+                    o = (int)m;
+        }
+    }
+    /* trace back from the cheapest last state with low bits o */
+    long s = ((long)choice[(size_t)(T - 1) * (size_t)nm + (size_t)o] << (L - K)) | o;
+    chunks[T - 1] = (unsigned char)(s & (nh - 1));
+    for (int i = T - 1; i > 0; --i) {
+        const long m = s >> K;
+        s = ((long)choice[(size_t)(i - 1) * (size_t)nm + (size_t)m] << (L - K)) | m;
+        chunks[i - 1] = (unsigned char)(s & (nh - 1));
+    }
+    *cost = prev[o];
+    *overlap = o;
+    free(prev);
+    free(next);
+    free(choice);
+    return 0;
+}
+
+/* Encodes a k x n fp32 matrix (row-major) into the trellis layout above: each
+ * tile's 256 targets in weight order i = 16 r + c go through
+ * oracle_encode_seq with L = 16, T = 256 and the codebook's values; chunk c_i
+ * fills stream positions [iK, iK + K), most significant bit first.  cost[t]
+ * is tile t's squared-error sum (tiles in [k/16][n/16] order).  OpenMP, when
+ * present, only splits the independent tiles. */
+int oracle_encode(const float *w, int64_t k, int64_t n, int K, uint16_t *trellis, float *cost, int threads)
+{
+    float *cb = (float *)malloc(sizeof(float) * 65536);
+    if (!cb)
+        return -1;
+    for (long st = 0; st < 65536; ++st)
+        cb[st] = (float)oracle_half_to_double(oracle_codebook((uint16_t)st));
+    const int64_t tn_count = n / 16, tiles = (k / 16) * tn_count;
+    int failed = 0;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(dynamic, 1) num_threads(threads > 0 ? threads : 1) reduction(| : failed)
+#endif
+    for (int64_t t = 0; t < tiles; ++t) {
+        float target[256];
+        unsigned char chunks[256];
+        const int64_t tk = t / tn_count, tn = t % tn_count;
+        for (int i = 0; i < 256; ++i)
+            target[i] = w[(tk * 16 + i / 16) * n + tn * 16 + i % 16];
+        int o = 0;
+        if (oracle_encode_seq(target, 256, 16, K, cb, chunks, &cost[t], &o) != 0) {
+            failed |= 1;
+            continue;
+        }
+        uint16_t *words = trellis + t * 16 * K;
+        memset(words, 0, sizeof(uint16_t) * 16 * (size_t)K);
+        for (int i = 0; i < 256; ++i)
+            for (int j = 0; j < K; ++j) {
+                const long p = (long)i * K + j;
+                if ((chunks[i] >> (K - 1 - j)) & 1)
+                    words[p / 16] |= (uint16_t)(1u << (15 - p % 16));
+            }
+    }
+    (void)threads;
+    free(cb);
+    return failed ? -1 : 0;
 }
 
 /* ------------------------------------------------------------ hadamard -- */
