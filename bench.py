@@ -43,12 +43,13 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-gemm", action="store_true", help="skip the m=2048 GEMM line item")
     ap.add_argument("--no-stack", action="store_true", help="skip the 70B layer-stack line items")
+    ap.add_argument("--no-encode", action="store_true", help="skip the trellis-encoder line item")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--profile", default=None,
                     help="profiling mode (no timing, no JSON): 'gemv-set' runs the decode GEMV set (one "
                          "exl3_gemv_multi call, as the bench step) warmup+steps times; 'gemm' runs the m=2048 prefill GEMM warmup+steps times; "
-                         "'gemv-layer:k:n:K' runs one m=1 layer")
+                         "'gemv-layer:k:n:K' runs one m=1 layer; 'encode' runs the trellis encoder on 256x256, K=4")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch without programmatic dependent launch (PDL is valid here: weights are immutable)")
     return ap.parse_args()
@@ -373,6 +374,9 @@ def run_ours(args, rank, world, local_rank):
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
 
     gemm_info = None
+    encode_info = None
+    if not args.no_encode:
+        encode_info = bench_encode(exl3, torch, stream)
     if not args.no_gemm:
         gemm_info = bench_gemm(exl3, torch, peaks, stream)
     stack_info = None
@@ -426,6 +430,8 @@ def run_ours(args, rank, world, local_rank):
                 "clocks": clocks}
         if gemm_info is not None:
             line["gemm"] = gemm_info
+        if encode_info is not None:
+            line["encode"] = encode_info
         if stack_info is not None:
             line["layer_stack"] = stack_info
         if not args.no_cpu_baseline and world == 1:
@@ -540,6 +546,36 @@ def bench_gemm(exl3, torch, peaks, stream):
             "peak_source": peaks["source"] + " bf16 cuBLAS burst (fp16 rate is the same)"}
 
 
+def bench_encode(exl3, torch, stream):
+    """Tail-biting trellis encoder (exl3_encode) on a 1024 x 1024 fp32 layer
+    (4096 tiles, targets ~N(0, 1.2^2)) at K = 4 and K = 2: tiles per second.
+    A tile is two Viterbi passes of 256 steps over 2^16 states."""
+    k = n = 1024
+    rng = np.random.default_rng(inputs.seed_for(5, 0))
+    w = torch.from_numpy((1.2 * rng.standard_normal((k, n))).astype(np.float32)).cuda()
+    out = []
+    for K in (4, 2):
+        ws = exl3.new_workspace(exl3.exl3_encode_workspace_size(k, n, K))
+        t = torch.empty((k // 16, n // 16, 16 * K), dtype=torch.uint16, device="cuda")
+        c = torch.empty((k // 16, n // 16), dtype=torch.float32, device="cuda")
+        with torch.cuda.stream(stream):
+            exl3.exl3_encode(w, K, trellis=t, cost=c, workspace=ws, stream=stream)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(2):
+                exl3.exl3_encode(w, K, trellis=t, cost=c, workspace=ws, stream=stream)
+            b.record(stream)
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / 2
+        tiles = (k // 16) * (n // 16)
+        out.append({"workload": "encode %dx%d fp32, K=%d" % (k, n, K), "ms": ms,
+                    "tiles_per_s": tiles / (ms * 1e-3),
+                    "state_updates_per_s": tiles * 2 * 256 * 65536 / (ms * 1e-3),
+                    "mse": float(c.sum()) / (k * n)})
+    return out
+
+
 def run_profile(args):
     """Launch-only mode for ncu: the same kernels as the timed run, no events."""
     import torch
@@ -551,7 +587,14 @@ def run_profile(args):
         exl3.exl3_set_launch_flags(exl3.EXL3_LAUNCH_PDL)
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
     what = args.profile
-    if what == "gemm":
+    if what == "encode":
+        # 256 x 256 fp32 (256 tiles), K = 4
+        rng = np.random.default_rng(inputs.seed_for(5, 0))
+        w = torch.from_numpy((1.2 * rng.standard_normal((256, 256))).astype(np.float32)).cuda()
+        ws = exl3.new_workspace(exl3.exl3_encode_workspace_size(256, 256, 4))
+        for _ in range(args.warmup + args.steps):
+            exl3.exl3_encode(w, 4, workspace=ws)
+    elif what == "gemm":
         m, k, n, K = 2048, 8192, 28672, 3
         L = inputs.make_layer(m, k, n, K, inputs.seed_for(3, 2))
         x, t, suh, svh = dev(L.x), dev(L.trellis), dev(L.suh), dev(L.svh)

@@ -202,6 +202,37 @@ exl3_status exl3_gemm(const void *x, const uint16_t *trellis, const void *suh, c
                       size_t workspace_bytes, void *stream);
 
 /*
+ * exl3_encode -- tail-biting trellis encoding of a weight matrix: for every
+ * 16 x 16 tile, the bit string whose decoded weights are closest in squared
+ * error to the tile's targets ([GEMM] section Viterbi编码内核剖析: a Viterbi
+ * forward pass over the trellis keeps the accumulated cost of every path and
+ * takes the cheapest; the tail-biting boundary is closed by enumerating start
+ * states, so the codeword's head and tail agree).  The inverse direction of
+ * exl3_decode_tiles: exl3_decode_tiles(exl3_encode(w)) is the encoded matrix.
+ *   w         k x n fp32, row-major: the target values (already in the
+ *             codebook's scale; the caller applies any scaling or rotation).
+ *   trellis   uint16 [k/16][n/16][16K] (output, layout above).
+ *   cost      (k/16) x (n/16) fp32 (output, nullable): each tile's sum of
+ *             squared errors, as the search computed it.
+ *   k, n      multiples of 16 (at most 2^22); K in [1, 8].
+ * The search (two passes per tile): pass 1 lets every state start and takes
+ * the low 16-K bits of the cheapest end as the overlap; pass 2 allows only
+ * starts whose high 16-K bits are that overlap and ends in the cheapest state
+ * whose low bits are it, then traces the path back.  Costs are fp32 (each
+ * weight's (w - cb(s))^2 added by one fused multiply-add), ties go to the
+ * smallest index; results are deterministic.
+ * `workspace` (at least exl3_encode_workspace_size bytes, device memory, no
+ * initialisation needed) holds the per-step choices of the CTAs in flight
+ * (256 x 2^(16-K) bytes per CTA, for up to ~1 GiB) and, for K = 1, their
+ * cost vectors.  Argument errors return EXL3_ERR_INVALID_ARG (null or
+ * misaligned w / trellis, bad sizes, w overlapping trellis) or
+ * EXL3_ERR_WORKSPACE before anything is launched.
+ */
+size_t exl3_encode_workspace_size(int64_t k, int64_t n, int K);
+exl3_status exl3_encode(const float *w, uint16_t *trellis, float *cost, int64_t k, int64_t n, int K,
+                        void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Launch options, process-wide (default 0).
  *
  * EXL3_LAUNCH_PDL -- launch exl3_gemv / exl3_gemm kernels with programmatic

@@ -141,3 +141,29 @@ def test_gemv_multi_argument_errors_and_sizes():
     many = [good] * 33
     assert size(many) >= size([good] * 32) + size([good])
     assert size([(A, B, C, D, E, 200, 256, 4)]) == 0
+
+
+def test_encode_argument_errors_and_sizes():
+    lib = exl3.load()
+    inv = exl3.EXL3_ERR_INVALID_ARG
+    ws = 1 << 24
+
+    def enc(w=A, t=B, cost=C, k=64, n=64, K=4, wsp=ws, wsb=1 << 40):
+        return lib.exl3_encode(w, t, cost, k, n, K, wsp, wsb, None)
+
+    assert enc(w=None) == inv
+    assert enc(t=MIS) == inv
+    assert enc(cost=A + 2) == inv            # fp32 costs need 4-byte alignment
+    assert enc(k=24) == inv                  # not a multiple of 16
+    assert enc(K=0) == inv and enc(K=9) == inv
+    assert enc(w=A, t=A) == inv              # trellis overlaps w
+    assert enc(wsp=None) == exl3.EXL3_ERR_WORKSPACE
+    assert enc(wsb=16) == exl3.EXL3_ERR_WORKSPACE
+    # per CTA in flight: 256 x 2^(16-K) bytes of recorded choices (plus the
+    # cost vectors for K = 1); never more CTAs than tiles
+    for K in range(1, 9):
+        one = lib.exl3_encode_workspace_size(16, 16, K)
+        extra = 2 * 4 * (1 << 15) if K == 1 else 0
+        assert one == 256 + 256 * (1 << (16 - K)) + extra
+        assert lib.exl3_encode_workspace_size(4096, 4096, K) <= 256 + (1 << 30)
+    assert lib.exl3_encode_workspace_size(24, 16, 4) == 0

@@ -25,6 +25,7 @@ EXPORTED = ["exl3_status_string", "exl3_version", "exl3_hadamard", "exl3_decode_
             "exl3_gemv_workspace_size", "exl3_gemv", "exl3_gemv_multi_workspace_size", "exl3_gemv_multi",
             "exl3_gemv_noalloc_max_scratch",
             "exl3_gemv_noalloc", "exl3_gemm_workspace_size", "exl3_gemm",
+            "exl3_encode_workspace_size", "exl3_encode",
             "exl3_workspace_status", "exl3_set_launch_flags", "exl3_launch_flags",
             "exl3_debug_set_wait_limit_ns", "exl3_debug_wait_limit_ns"]
 
@@ -85,6 +86,10 @@ def load(build_if_needed=True):
         lib.exl3_gemv_noalloc_max_scratch.restype = sz
         lib.exl3_gemv_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, ci, vp]
         lib.exl3_gemv_noalloc.restype = ci
+        lib.exl3_encode_workspace_size.argtypes = [i64, i64, ci]
+        lib.exl3_encode_workspace_size.restype = sz
+        lib.exl3_encode.argtypes = [vp, vp, vp, i64, i64, ci, vp, sz, vp]
+        lib.exl3_encode.restype = ci
         lib.exl3_workspace_status.argtypes = [vp, sz, ci, vp]
         lib.exl3_workspace_status.restype = ci
         lib.exl3_set_launch_flags.argtypes = [ctypes.c_uint]
@@ -258,6 +263,28 @@ def exl3_gemv_noalloc(x, trellis, suh, svh, K, y, stream=None):
 def exl3_gemm(x, trellis, suh, svh, K, y=None, workspace=None, stream=None):
     """The same layer on the tensor cores, any m (tuned for m >= 64)."""
     return _linear(load().exl3_gemm, "exl3_gemm", x, trellis, suh, svh, K, y, workspace, stream)
+
+
+def exl3_encode_workspace_size(k, n, K):
+    return int(load().exl3_encode_workspace_size(k, n, K))
+
+
+def exl3_encode(w, K, trellis=None, cost=None, workspace=None, stream=None):
+    """Tail-biting trellis encoding of a k x n fp32 matrix into a [k/16, n/16, 16K]
+    uint16 trellis.  Returns (trellis, cost): cost[tk, tn] is the tile's fp32
+    squared-error sum."""
+    k, n = w.shape
+    if trellis is None:
+        trellis = torch.empty((k // 16, n // 16, 16 * K), dtype=torch.uint16, device=w.device)
+    if cost is None:
+        cost = torch.empty((k // 16, n // 16), dtype=torch.float32, device=w.device)
+    if workspace is None:
+        raise ValueError("exl3_encode needs a workspace (see new_workspace / exl3_encode_workspace_size)")
+    _check(load().exl3_encode(_dev(w, torch.float32, "w"), _dev(trellis, torch.uint16, "trellis"),
+                              _dev(cost, torch.float32, "cost"), k, n, int(K),
+                              _dev(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)),
+           "exl3_encode")
+    return trellis, cost
 
 
 def exl3_workspace_status(workspace, clear=False, stream=None):
