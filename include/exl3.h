@@ -233,6 +233,48 @@ exl3_status exl3_encode(const float *w, uint16_t *trellis, float *cost, int64_t 
                         void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * exl3_udu -- block factorisation H = U D U^T of a symmetric positive
+ * definite k x k matrix (fp64), 16 x 16 blocks: U unit block-upper-triangular,
+ * D block-diagonal ([GEMM] section Viterbi编码内核剖析: ldlq() performs a
+ * block-wise LDL decomposition before the trellis encoding).
+ *   h         k x k fp64, row-major (read; may equal ud).
+ *   ud        k x k fp64 (output): the diagonal blocks hold D_b, the strictly
+ *             upper blocks U_ab (a < b), the strictly lower blocks are zero.
+ *   k         multiple of 16, at most 65536.
+ *   workspace at least exl3_udu_workspace_size(k) bytes of device memory.
+ * Bottom-up: D_b = H_bb - sum_{c>b} U_bc D_c U_bc^T, U_ab = (H_ab - sum_{c>b}
+ * U_ac D_c U_bc^T) D_b^-1 (D_b inverted by Gauss-Jordan without pivoting), all
+ * in fp64.  EXL3_ERR_INVALID_ARG for null or misaligned pointers, bad k, or h
+ * and ud overlapping without being equal.
+ */
+size_t exl3_udu_workspace_size(int64_t k);
+exl3_status exl3_udu(const double *h, double *ud, int64_t k, void *workspace, size_t workspace_bytes,
+                     void *stream);
+
+/*
+ * exl3_ldlq -- Hessian-aware trellis quantisation of a layer (LDLQ with the
+ * trellis encoder; [GEMM] section Viterbi编码内核剖析: ldlq() decomposes the
+ * Hessian block-wise, then the trellis kernel encodes the 16 x 16 tiles).
+ *   w         k x n fp32, row-major: the layer in the x . W orientation (rows
+ *             = input channels).
+ *   h         k x k fp64: the input Hessian (symmetric positive definite).
+ *   trellis   uint16 [k/16][n/16][16K] (output).
+ *   w_hat     k x n fp32 (output, nullable): the decoded weights.
+ *   k         multiple of 16 (at most 65536); n multiple of 16; K in [1, 8].
+ * With H = U D U^T (exl3_udu), tile rows are encoded in order: row block b's
+ * target T_b = W_b - sum_{c<b} U_{c,b}^T (W_hat_c - W_c) is formed in fp64,
+ * rounded to fp32 and encoded (exl3_encode), so that the proxy loss
+ * tr((W_hat - W)^T H (W_hat - W)) is sum_b tr(F_b^T D_b F_b), F_b = W_hat_b -
+ * T_b.  With H = I (or any block-diagonal H) this is exl3_encode of W.
+ * `workspace`: at least exl3_ldlq_workspace_size bytes (the factor, the
+ * errors and the encoder's workspace; no initialisation needed).  Argument
+ * errors as exl3_encode (w_hat must not overlap w or trellis).
+ */
+size_t exl3_ldlq_workspace_size(int64_t k, int64_t n, int K);
+exl3_status exl3_ldlq(const float *w, const double *h, uint16_t *trellis, float *w_hat, int64_t k, int64_t n,
+                      int K, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Launch options, process-wide (default 0).
  *
  * EXL3_LAUNCH_PDL -- launch exl3_gemv / exl3_gemm kernels with programmatic

@@ -167,3 +167,28 @@ def test_encode_argument_errors_and_sizes():
         assert one == 256 + 256 * (1 << (16 - K)) + extra
         assert lib.exl3_encode_workspace_size(4096, 4096, K) <= 256 + (1 << 30)
     assert lib.exl3_encode_workspace_size(24, 16, 4) == 0
+
+
+def test_udu_and_ldlq_argument_errors_and_sizes():
+    lib = exl3.load()
+    inv = exl3.EXL3_ERR_INVALID_ARG
+    assert lib.exl3_udu(None, B, 32, C, 1 << 20, None) == inv
+    assert lib.exl3_udu(A, B, 24, C, 1 << 20, None) == inv          # not a multiple of 16
+    assert lib.exl3_udu(A, A + 64, 32, C, 1 << 20, None) == inv     # overlapping, not equal
+    assert lib.exl3_udu(A, B, 32, None, 0, None) == exl3.EXL3_ERR_WORKSPACE
+    assert lib.exl3_udu_workspace_size(32) == 256 + 16 * 16 * 8 + 32 * 16 * 8
+    assert lib.exl3_udu_workspace_size(24) == 0
+
+    def ldlq(w=A, h=B, t=C, wh=None, k=64, n=64, K=4, ws=D, wsb=1 << 40):
+        return lib.exl3_ldlq(w, h, t, wh, k, n, K, ws, wsb, None)
+
+    assert ldlq(w=None) == inv
+    assert ldlq(h=MIS) == inv
+    assert ldlq(K=9) == inv
+    assert ldlq(n=40) == inv
+    assert ldlq(wh=A) == inv                                         # w_hat overlaps w
+    assert ldlq(ws=None) == exl3.EXL3_ERR_WORKSPACE
+    # the factor and the errors in fp64, plus the encoder's workspace for 16 x n
+    need = lib.exl3_ldlq_workspace_size(64, 128, 4)
+    assert need >= 64 * 64 * 8 + 64 * 128 * 8 + lib.exl3_encode_workspace_size(16, 128, 4)
+    assert lib.exl3_ldlq_workspace_size(64, 40, 4) == 0

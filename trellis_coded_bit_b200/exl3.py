@@ -25,7 +25,8 @@ EXPORTED = ["exl3_status_string", "exl3_version", "exl3_hadamard", "exl3_decode_
             "exl3_gemv_workspace_size", "exl3_gemv", "exl3_gemv_multi_workspace_size", "exl3_gemv_multi",
             "exl3_gemv_noalloc_max_scratch",
             "exl3_gemv_noalloc", "exl3_gemm_workspace_size", "exl3_gemm",
-            "exl3_encode_workspace_size", "exl3_encode",
+            "exl3_encode_workspace_size", "exl3_encode", "exl3_udu_workspace_size", "exl3_udu",
+            "exl3_ldlq_workspace_size", "exl3_ldlq",
             "exl3_workspace_status", "exl3_set_launch_flags", "exl3_launch_flags",
             "exl3_debug_set_wait_limit_ns", "exl3_debug_wait_limit_ns"]
 
@@ -90,6 +91,14 @@ def load(build_if_needed=True):
         lib.exl3_encode_workspace_size.restype = sz
         lib.exl3_encode.argtypes = [vp, vp, vp, i64, i64, ci, vp, sz, vp]
         lib.exl3_encode.restype = ci
+        lib.exl3_udu_workspace_size.argtypes = [i64]
+        lib.exl3_udu_workspace_size.restype = sz
+        lib.exl3_udu.argtypes = [vp, vp, i64, vp, sz, vp]
+        lib.exl3_udu.restype = ci
+        lib.exl3_ldlq_workspace_size.argtypes = [i64, i64, ci]
+        lib.exl3_ldlq_workspace_size.restype = sz
+        lib.exl3_ldlq.argtypes = [vp, vp, vp, vp, i64, i64, ci, vp, sz, vp]
+        lib.exl3_ldlq.restype = ci
         lib.exl3_workspace_status.argtypes = [vp, sz, ci, vp]
         lib.exl3_workspace_status.restype = ci
         lib.exl3_set_launch_flags.argtypes = [ctypes.c_uint]
@@ -285,6 +294,39 @@ def exl3_encode(w, K, trellis=None, cost=None, workspace=None, stream=None):
                               _dev(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)),
            "exl3_encode")
     return trellis, cost
+
+
+def exl3_udu(h, ud=None, stream=None):
+    """Block factorisation H = U D U^T (fp64, 16 x 16 blocks) of a k x k CUDA
+    tensor: returns ud with D in the diagonal blocks, U above them, zeros below."""
+    k = h.shape[0]
+    if ud is None:
+        ud = torch.empty_like(h)
+    ws = new_workspace(load().exl3_udu_workspace_size(k), device=h.device)
+    _check(load().exl3_udu(_dev(h, torch.float64, "h"), _dev(ud, torch.float64, "ud"), k,
+                           _dev(ws, torch.uint8, "workspace"), ws.numel(), _stream(stream)), "exl3_udu")
+    return ud
+
+
+def exl3_ldlq_workspace_size(k, n, K):
+    return int(load().exl3_ldlq_workspace_size(k, n, K))
+
+
+def exl3_ldlq(w, h, K, trellis=None, w_hat=None, workspace=None, stream=None):
+    """LDLQ of a k x n fp32 layer against the k x k fp64 Hessian h with the
+    K-bit trellis encoder.  Returns (trellis, w_hat)."""
+    k, n = w.shape
+    if trellis is None:
+        trellis = torch.empty((k // 16, n // 16, 16 * K), dtype=torch.uint16, device=w.device)
+    if w_hat is None:
+        w_hat = torch.empty((k, n), dtype=torch.float32, device=w.device)
+    if workspace is None:
+        raise ValueError("exl3_ldlq needs a workspace (see new_workspace / exl3_ldlq_workspace_size)")
+    _check(load().exl3_ldlq(_dev(w, torch.float32, "w"), _dev(h, torch.float64, "h"),
+                            _dev(trellis, torch.uint16, "trellis"), _dev(w_hat, torch.float32, "w_hat"), k, n,
+                            int(K), _dev(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)),
+           "exl3_ldlq")
+    return trellis, w_hat
 
 
 def exl3_workspace_status(workspace, clear=False, stream=None):
