@@ -377,6 +377,7 @@ def run_ours(args, rank, world, local_rank):
     encode_info = None
     if not args.no_encode:
         encode_info = bench_encode(exl3, torch, stream)
+        encode_info.append(bench_ldlq(exl3, torch, stream))
     if not args.no_gemm:
         gemm_info = bench_gemm(exl3, torch, peaks, stream)
     stack_info = None
@@ -574,6 +575,42 @@ def bench_encode(exl3, torch, stream):
                     "state_updates_per_s": tiles * 2 * 256 * 65536 / (ms * 1e-3),
                     "mse": float(c.sum()) / (k * n)})
     return out
+
+
+def bench_ldlq(exl3, torch, stream):
+    """LDLQ (exl3_ldlq) of a 1024 x 4096 fp32 layer, K = 4, against a synthetic
+    correlated Hessian (inputs x = z C, neighbouring channels correlated with
+    rho = 0.95, plus a 0.1% ridge): time, and the proxy loss tr(E^T H E)
+    relative to encoding the layer without feedback (exl3_encode)."""
+    k, n, K = 1024, 4096, 4
+    rng = np.random.default_rng(inputs.seed_for(5, 1))
+    w = torch.from_numpy(rng.standard_normal((k, n)).astype(np.float32)).cuda()
+    idx = np.arange(k)
+    c = 0.95 ** np.abs(idx[:, None] - idx[None, :])
+    x = rng.standard_normal((4 * k, k)) @ np.linalg.cholesky(c).T
+    hn = x.T @ x / x.shape[0]
+    hn += 1e-3 * np.trace(hn) / k * np.eye(k)
+    h = torch.from_numpy(hn).cuda()
+    ws = exl3.new_workspace(exl3.exl3_ldlq_workspace_size(k, n, K))
+    with torch.cuda.stream(stream):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        _, w_hat = exl3.exl3_ldlq(w, h, K, workspace=ws, stream=stream)
+        b.record(stream)
+        ews = exl3.new_workspace(exl3.exl3_encode_workspace_size(k, n, K))
+        plain, _ = exl3.exl3_encode(w, K, workspace=ews, stream=stream)
+        p_hat = exl3.exl3_decode_tiles(plain, k, n, K, stream=stream).float()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+
+    def loss(wh):
+        e = (wh.double() - w.double())
+        return float((e * (h @ e)).sum())
+
+    return {"workload": "LDLQ 1024x4096 fp32, K=4, correlated synthetic Hessian", "ms": ms,
+            "tiles_per_s": (k // 16) * (n // 16) / (ms * 1e-3),
+            "proxy_loss_vs_plain_encoding": loss(w_hat) / loss(p_hat)}
 
 
 def run_profile(args):
