@@ -420,24 +420,25 @@ __device__ __forceinline__ void gemv_cta(const GemvParams &p, const GemvGroup &g
     for (int mg = 0; mg < MG; ++mg)
         act_live[mg] = 8 * mg + ((lane >> 1) & 7) < m;
 
-    // this warp's units: u0 + warp + 8i, i < nunits
-    const int nunits = u0 + warp < u1 ? (int)((u1 - u0 - warp + 7) >> 3) : 0;
+    // this warp's units: u0 + warp + kGemvWarps i, i < nunits
+    const int nunits = u0 + warp < u1 ? (int)((u1 - u0 - warp + kGemvWarps - 1) / kGemvWarps) : 0;
 
     // issue iterator (runs kGemvDepth units ahead of consumption): the next
     // unit to copy is at (layer il, column block icb, tile row itr); `rem`
-    // units are left to copy
+    // units are left to copy.  A step of kGemvWarps tile rows crosses at most
+    // one column block while kGemvWarps <= every layer's tile rows (k >= 128)
     int rem = nunits;
     int il = lb, icb = 0, itr = 0;
     gemv_locate(p, le, rem ? u0 + warp : u0, il, icb, itr);
     int itr_lim = 0, incb = 0;
-    int64_t tile_rows8 = 0;  // 8 tile rows of the layer's matrix, in bytes
+    int64_t tile_rows_step = 0;  // kGemvWarps tile rows of the layer's matrix, in bytes
     const unsigned char *isrc = nullptr, *iasrc = nullptr;
     auto enter_block = [&]() {
         const GemvLayer &L = p.L[il];
         itr_lim = L.tr_count;
         incb = L.n >> 7;
         const int64_t tile_row_bytes = (int64_t)(L.n >> 4) * 32 * K;
-        tile_rows8 = kGemvWarps * tile_row_bytes;
+        tile_rows_step = kGemvWarps * tile_row_bytes;
         isrc = L.trellis + itr * tile_row_bytes + (int64_t)icb * 256 * K + lane * 16;
         iasrc = L.acts + (int64_t)itr * MG * kGemvActBlock + lane * 16;
     };
@@ -459,7 +460,7 @@ __device__ __forceinline__ void gemv_cta(const GemvParams &p, const GemvGroup &g
             if (r < kTrChunks - 1 || last_chunk)
                 cp_async16(tdst[r] + so, isrc + 512 * r);
         --rem;
-        isrc += tile_rows8;
+        isrc += tile_rows_step;
         iasrc += kGemvWarps * MG * kGemvActBlock;
         itr += kGemvWarps;
         if (itr >= itr_lim) {  // next column block, perhaps of the next layer (8 <= every TR)
@@ -534,7 +535,7 @@ __device__ __forceinline__ void gemv_cta(const GemvParams &p, const GemvGroup &g
         const int64_t blk_begin = SL.unit_begin + (int64_t)cbk * TR, blk_end = blk_begin + TR;
         const int64_t seg_begin = blk_begin > u0 ? blk_begin : u0;
         const int64_t seg_end = blk_end < u1 ? blk_end : u1;
-        // this warp's units below seg_end: ceil((seg_end - u0 - warp) / 8)
+        // this warp's units below seg_end: ceil((seg_end - u0 - warp) / kGemvWarps)
         const int rel_end = (int)(seg_end - u0) - warp;
         const int upto = rel_end > 0 ? (rel_end + kGemvWarps - 1) / kGemvWarps : 0;
         for (; ci < upto; ++ci) {
