@@ -26,8 +26,9 @@
 //   * M ping-pongs in shared memory (2 x 2^(16-K) fp32, up to 128 KB at K = 2,
 //     so smaller K leave room for more CTAs per SM); for K = 1 it would need
 //     256 KB and lives in the CTA's workspace slot instead (L2);
-//   * the codebook value of a state is computed on the fly (one IMAD, one
-//     LOP3, an fp16 add), as in the decode;
+//   * the codebook value of a state is computed on the fly, as in the decode
+//     (the multiply stepped by one add across an entry's states, one LOP3,
+//     an fp16 add);
 //   * the recorded choices (one byte per entry and weight) go to the CTA's
 //     workspace slot; one thread traces back, then the CTA packs the 16K
 //     words in parallel.
@@ -50,38 +51,37 @@ struct EncShape {
     static constexpr size_t kSmem = (kGlobalM ? 0 : (size_t)2 * NM * 4) + 256 * 4 + 256 + 2 * 32 * 8;
 };
 
-// Codebook value of a 16-bit state as fp32: the fp16 sum (round to nearest
-// even) of the two fp16 halves of the masked product, exactly as the decode
-// forms it.
-__device__ __forceinline__ float enc_codebook(uint32_t s, const Codebook &cb)
-{
-    const uint32_t v = codebook_word(s, cb);
-    const __half2 h = *reinterpret_cast<const __half2 *>(&v);
-    return __half2float(__hadd(__low2half(h), __high2half(h)));
-}
-
 // One step of the recursion over the thread's entries: prev -> next, choices
-// to `choice` (a row of NM bytes) when RECORD.
+// to `choice` (a row of NM bytes) when RECORD.  The states of an entry m are
+// s_h = (h << (16-K)) | m = m + h 2^(16-K), so their codebook products are
+// v_h = v_0 + h (C1 << (16-K)) (mod 2^32), one add per state, and their
+// predecessor costs sit at prev[(m >> K) + h 2^(16-2K)]: a per-m base plus a
+// per-h constant offset.  The integer values are the same as in the plain
+// formula, so the decisions are unchanged.
 template <int K, bool RECORD>
 __device__ __forceinline__ void enc_step(float wi, const float *prev, float *next, unsigned char *choice,
-                                         const Codebook &cb)
+                                         const Codebook &cb, uint32_t dv)
 {
     using Sh = EncShape<K>;
     const int j = threadIdx.x;
 #pragma unroll 2
     for (int q = 0; q < Sh::PER; ++q) {
         const uint32_t m = (uint32_t)(j + kEncThreads * q);
+        const float *pm = prev + (m >> K);
+        uint32_t v = m * cb.mul + cb.add;
         float best = 0.f;
         int best_h = 0;
 #pragma unroll(K <= 4 ? (1 << K) : 4)
         for (int h = 0; h < (1 << K); ++h) {
-            const uint32_t s = ((uint32_t)h << (16 - K)) | m;
-            const float d = wi - enc_codebook(s, cb);
-            const float v = __fmaf_rn(d, d, prev[s >> K]);
-            if (h == 0 || v < best) {
-                best = v;
+            const uint32_t w = (v & cb.mask) ^ cb.xr;
+            const __half2 hw = *reinterpret_cast<const __half2 *>(&w);
+            const float d = wi - __half2float(__hadd(__low2half(hw), __high2half(hw)));
+            const float val = __fmaf_rn(d, d, pm[h << (16 - 2 * K)]);
+            if (h == 0 || val < best) {
+                best = val;
                 best_h = h;
             }
+            v += dv;
         }
         next[m] = best;
         if (RECORD)
@@ -113,6 +113,7 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(const float *__rest
     int *red_i = reinterpret_cast<int *>(red_v + 32);
     const int j = threadIdx.x, lane = j & 31, warp = j >> 5;
     const int64_t tn_count = n / 16, tiles = (k / 16) * tn_count;
+    const uint32_t dv = cb.mul << (16 - K);  // codebook-product step from state s to s + 2^(16-K)
 
     for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
         const int64_t tk = tile / tn_count, tn = tile - tk * tn_count;
@@ -127,9 +128,9 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(const float *__rest
             __syncthreads();
             for (int i = 0; i < 256; ++i) {
                 if (pass == 1)
-                    enc_step<K, false>(target[i], prev, next, nullptr, cb);
+                    enc_step<K, false>(target[i], prev, next, nullptr, cb, dv);
                 else
-                    enc_step<K, true>(target[i], prev, next, choices + (size_t)i * NM, cb);
+                    enc_step<K, true>(target[i], prev, next, choices + (size_t)i * NM, cb, dv);
                 __syncthreads();
                 float *t = prev;
                 prev = next;
