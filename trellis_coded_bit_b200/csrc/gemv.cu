@@ -6,19 +6,22 @@
 // B200 design (the pages' consumer-GPU GEMV is prior art, not copied):
 //   * Two launches.  A rotation kernel computes x' = H(x .* suh)/sqrt(128)
 //     (fp32 butterflies, fp16 result) and writes it into the workspace as
-//     tensor-core B-fragment activation blocks (see below).  The main kernel then has
-//     no prologue: every warp starts streaming weights at once.
-//   * The main kernel is persistent and "stream-K" balanced at warp level:
-//     the work units are (layer, 128-column block, tile row of 16 input
-//     channels), numbered consecutively over every layer of the launch (any
-//     mix of K), and warp w of W owns the contiguous range [wU/W, (w+1)U/W)
-//     -- every warp gets the same amount of work, whatever the shapes.  A
-//     range is cut into segments at column-block boundaries.  At a segment end
-//     the warp writes its fp32 partial of the block to the workspace; the last
-//     warp to arrive on the block's counter (atomic ticket, no spinning) sums
-//     the block's partials in a fixed order (deterministic) and finishes it
-//     (output rotation, svh, fp16 y).  Warps never wait for one another, and
-//     one launch serves all the layers of an exl3_gemv_multi call.
+//     tensor-core B-fragment activation blocks (see below); the main kernel
+//     streams the weights and copies those blocks with them.
+//   * The main kernel is persistent and "stream-K" balanced.  One launch
+//     serves every layer of an exl3_gemv_multi call (up to 32, any mix of K):
+//     its CTAs are split into one group per K, in proportion to the group's
+//     cost, so that each CTA runs the decode compiled for one K.  Within a
+//     group the work units -- (layer, 128-column block, tile row of 16 input
+//     channels) -- are numbered consecutively and CTA c of G owns the
+//     contiguous range [cU/G, (c+1)U/G); its 8 warps take units u0 + w,
+//     u0 + w + 8, ..., so a CTA's concurrent loads stay within a few
+//     consecutive tile rows.  A range is cut into segments at column-block
+//     boundaries.  At a segment end the warps' partials meet in shared memory
+//     (one barrier) and either finish the block (output rotation, svh, fp16 y)
+//     or go to the workspace, where the last segment to arrive on the block's
+//     counter (atomic ticket, no spinning) sums all segments in segment order
+//     (deterministic) and finishes it.
 //   * The MAC runs on the tensor cores (mma.sync m16n8k16, fp32 accumulate)
 //     with the WEIGHTS in the A operand: a codebook word's two fp16 halves
 //     form a pair of k slots and the activation is duplicated over that pair
@@ -159,10 +162,10 @@ struct GemvGroup {
 // launch parameters so that they stay opaque registers: a multiply by a
 // register runs on the FMA pipe (IMAD), which the decode leaves half idle,
 // while shifts and byte permutes compete with the codebook's LOP3 for the
-// ALU pipe.  pow2[i] = 2^i, hi16 = 2^16 (mul.hi by it is a right shift by 16).
+// ALU pipe.  pow2[i] = 2^i.  (The upper-half word windows stay byte permutes:
+// as a mul.hi by 2^16 they measured slower.)
 struct GemvMults {
     uint32_t pow2[8];
-    uint32_t hi16;
 };
 
 struct GemvParams {
@@ -223,8 +226,9 @@ __device__ __forceinline__ void cp_async_wait()
 // multiple of 16 the window is the word W'[e/16 - 1]; otherwise it lies in
 // V = W'[a-1]:W'[a] (a = e / 16, as one big-endian 32-bit value) shifted
 // right by c = 16 - e % 16, and is one byte permute with zero fill of V or of
-// V pre-shifted by c % 8.  All selectors are compile-time constants, and the
-// V values and their shifted copies are shared between windows.
+// V times 2^(8 - c % 8) (a left shift, as a multiply on the FMA pipe).  All
+// selectors are compile-time constants, and the V values and their shifted
+// copies are shared between windows.
 template <int K>
 __device__ __forceinline__ void pair_states(const uint32_t (&R)[K + 1], uint32_t (&s)[32], const GemvMults &mu)
 {
@@ -234,11 +238,7 @@ __device__ __forceinline__ void pair_states(const uint32_t (&R)[K + 1], uint32_t
         const int a = e >> 4, rb = e & 15;
         if (rb == 0) {
             const int w = a - 1;
-#if GEMV_WORD_HI_IMAD
-            s[jj] = (w & 1) ? __byte_perm(R[(w + 1) >> 1], 0u, 0x4410u) : __umulhi(R[w >> 1], mu.hi16);
-#else
             s[jj] = (w & 1) ? __byte_perm(R[(w + 1) >> 1], 0u, 0x4410u) : __byte_perm(R[w >> 1], 0u, 0x4432u);
-#endif
         } else {
             const uint32_t v = (a & 1) ? __byte_perm(R[(a - 1) >> 1], R[(a + 1) >> 1], 0x3254u)
                                        : __byte_perm(R[a >> 1], 0u, 0x1032u);
@@ -901,7 +901,6 @@ static exl3_status run_gemv_launch(const exl3_linear *const *layers, int count, 
     p.cb = codebook_constants();
     for (int i = 0; i < 8; ++i)
         p.mu.pow2[i] = 1u << i;
-    p.mu.hi16 = 1u << 16;
     for (int i = 0; i < count; ++i) {
         const int l = pl.order[i];
         GemvLayer &L = p.L[i];
