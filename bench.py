@@ -326,6 +326,22 @@ def run_ours(args, rank, world, local_rank):
         total_ms = max_over_ranks(total_ms, dist)
         dist.barrier()
 
+    # spread of the step time: each replay bracketed by its own events (after
+    # the timed region, so the contract's number is untouched)
+    step_us = []
+    with torch.cuda.stream(stream):
+        pairs = []
+        for _ in range(max(20, args.steps)):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            graph.replay()
+            b.record(stream)
+            pairs.append((a, b))
+    torch.cuda.synchronize()
+    step_us = sorted(a.elapsed_time(b) * 1e3 for a, b in pairs)
+    pct = lambda q: step_us[min(len(step_us) - 1, int(q * len(step_us)))]
+
     # the same 20 layers as 20 exl3_gemv calls (one graph), for comparison
     with torch.cuda.stream(stream):
         for _ in range(3):
@@ -420,6 +436,7 @@ def run_ours(args, rank, world, local_rank):
                           "gemv_kernel whose CTAs are split into K groups (%d launch pair(s)); duration = timed "
                           "region / steps (one CUDA-graph replay per step)" % n_launches,
                 "peak_source": peaks["source"] + " (burst copy)",
+                "step_us_p10_p50_p90": [pct(0.1), pct(0.5), pct(0.9)],
                 "decode_view": {"weights_per_clk_per_sm": w_clk_sm,
                                 "alu_ceiling_weights_per_clk_per_sm": ALU_CEILING_WEIGHTS_PER_CLK_PER_SM,
                                 "frac_of_alu_ceiling": w_clk_sm / ALU_CEILING_WEIGHTS_PER_CLK_PER_SM,

@@ -81,3 +81,36 @@ def test_multi_is_deterministic():
         torch.cuda.synchronize()
         for y, z in zip(ys, again):
             assert np.array_equal(y, z.cpu().numpy().astype(np.float64))
+
+
+def test_multi_with_views_into_contiguous_buffers():
+    # x and y of every layer are views into one device buffer each (as an
+    # application batching a decode step's activations would hold them)
+    shapes = [(256, 384, 3), (1024, 128, 2), (128, 256, 8), (384, 640, 4)]
+    layers = [inputs.make_layer(2, k, n, K, seed=8700 + i) for i, (k, n, K) in enumerate(shapes)]
+    ref, _, _ = run_multi(layers)
+    xs = torch.cat([dev(L.x).reshape(-1) for L in layers])
+    ys = torch.empty(sum(2 * L.n for L in layers), dtype=torch.float16, device="cuda")
+    args, ox, oy = [], 0, 0
+    for L in layers:
+        xv = xs[ox:ox + 2 * L.k].view(2, L.k)
+        yv = ys[oy:oy + 2 * L.n].view(2, L.n)
+        args.append((xv, dev(L.trellis), dev(L.suh), dev(L.svh), L.K, yv))
+        ox += 2 * L.k
+        oy += 2 * L.n
+    ws = exl3.new_workspace(exl3.exl3_gemv_multi_workspace_size(args, 2))
+    exl3.exl3_gemv_multi(args, workspace=ws)
+    torch.cuda.synchronize()
+    for a, r in zip(args, ref):
+        assert np.array_equal(a[5].cpu().numpy().astype(np.float64), r)
+
+
+@pytest.mark.parametrize("m", [1, 12])
+def test_multi_tiny_and_large_k_groups(m):
+    # a one-block K = 1 layer (8 units: its CTA group is a single CTA) beside a
+    # large K = 8 layer that takes the rest of the grid
+    layers = [inputs.make_layer(m, 128, 128, 1, seed=8800 + m), inputs.make_layer(m, 2048, 2048, 8, seed=8900 + m)]
+    ys, _, _ = run_multi(layers)
+    check(layers[0], ys[0])
+    check(layers[1], ys[1], col_blocks=(0, 2))
+    check(layers[1], ys[1], col_blocks=(14, 16))
