@@ -49,7 +49,8 @@ def parse():
     ap.add_argument("--profile", default=None,
                     help="profiling mode (no timing, no JSON): 'gemv-set' runs the decode GEMV set (one "
                          "exl3_gemv_multi call, as the bench step) warmup+steps times; 'gemm' runs the m=2048 prefill GEMM warmup+steps times; "
-                         "'gemv-layer:k:n:K' runs one m=1 layer; 'encode' runs the trellis encoder on 256x256, K=4")
+                         "'gemv-layer:k:n:K' runs one m=1 layer; 'gemm:m:k:n:K' runs one GEMM shape; 'encode' runs the trellis "
+                         "encoder on 256x256, K=4")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch without programmatic dependent launch (PDL is valid here: weights are immutable)")
     return ap.parse_args()
@@ -665,6 +666,15 @@ def run_profile(args):
         ws = exl3.new_workspace(exl3.exl3_encode_workspace_size(256, 256, 4))
         for _ in range(args.warmup + args.steps):
             exl3.exl3_encode(w, 4, workspace=ws)
+    elif what.startswith("gemm:"):
+        # one GEMM shape, random trellis: gemm:m:k:n:K
+        _, m, k, n, K = what.split(":")
+        m, k, n, K = int(m), int(k), int(n), int(K)
+        L = inputs.make_layer(m, k, n, K, seed=2)
+        x, t, suh, svh = dev(L.x), dev(L.trellis), dev(L.suh), dev(L.svh)
+        ws = exl3.new_workspace(exl3.exl3_gemm_workspace_size(m, k, n, K))
+        for _ in range(args.warmup + args.steps):
+            exl3.exl3_gemm(x, t, suh, svh, K, workspace=ws)
     elif what == "gemm":
         m, k, n, K = 2048, 8192, 28672, 3
         L = inputs.make_layer(m, k, n, K, inputs.seed_for(3, 2))
