@@ -225,8 +225,8 @@ exl3_status exl3_gemm(const void *x, const uint16_t *trellis, const void *suh, c
  * initialisation needed) holds the per-step choices of the CTAs in flight
  * (256 x 2^(16-K) bytes per CTA, for up to ~1 GiB) and, for K = 1, their
  * cost vectors.  Argument errors return EXL3_ERR_INVALID_ARG (null or
- * misaligned w / trellis, bad sizes, w overlapping trellis) or
- * EXL3_ERR_WORKSPACE before anything is launched.
+ * misaligned w / trellis, bad sizes, any two of w, trellis and cost
+ * overlapping) or EXL3_ERR_WORKSPACE before anything is launched.
  */
 size_t exl3_encode_workspace_size(int64_t k, int64_t n, int K);
 exl3_status exl3_encode(const float *w, uint16_t *trellis, float *cost, int64_t k, int64_t n, int K,

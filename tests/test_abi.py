@@ -157,6 +157,8 @@ def test_encode_argument_errors_and_sizes():
     assert enc(k=24) == inv                  # not a multiple of 16
     assert enc(K=0) == inv and enc(K=9) == inv
     assert enc(w=A, t=A) == inv              # trellis overlaps w
+    assert enc(cost=A + 64) == inv           # cost overlaps w
+    assert enc(cost=B) == inv                # cost overlaps trellis
     assert enc(wsp=None) == exl3.EXL3_ERR_WORKSPACE
     assert enc(wsb=16) == exl3.EXL3_ERR_WORKSPACE
     # per CTA in flight: 256 x 2^(16-K) bytes of recorded choices (plus the

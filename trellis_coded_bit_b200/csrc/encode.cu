@@ -285,7 +285,10 @@ extern "C" exl3_status exl3_encode(const float *w, uint16_t *trellis, float *cos
         return EXL3_ERR_INVALID_ARG;
     if (!enc_args_ok(k, n, K))
         return EXL3_ERR_INVALID_ARG;
-    if (ranges_overlap(w, (size_t)(k * n * 4), trellis, (size_t)(k * n * K / 8)))
+    const size_t cost_bytes = (size_t)((k / 16) * (n / 16)) * 4;
+    if (ranges_overlap(w, (size_t)(k * n * 4), trellis, (size_t)(k * n * K / 8)) ||
+        (cost && (ranges_overlap(cost, cost_bytes, w, (size_t)(k * n * 4)) ||
+                  ranges_overlap(cost, cost_bytes, trellis, (size_t)(k * n * K / 8)))))
         return EXL3_ERR_INVALID_ARG;
     EncPlan pl;
     enc_plan(K, (k / 16) * (n / 16), pl);
