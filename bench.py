@@ -200,6 +200,52 @@ def cpu_oracle_sample(layers, seconds):
             "seconds": spent}
 
 
+def cpu_oracle_one_thread(layers, seconds):
+    """The single-threaded oracle (the parity configuration) on one 128-column
+    block per layer call, round-robin until ~`seconds`."""
+    import oracle
+
+    done_bytes, spent, i = 0, 0.0, 0
+    t_end = time.perf_counter() + seconds
+    while time.perf_counter() < t_end and i < 2 * len(layers):
+        L = layers[i % len(layers)]
+        b0 = (i // len(layers)) % (L.n // 128)
+        t0 = time.perf_counter()
+        oracle.linear(L.x, L.trellis, L.suh, L.svh, L.K, col_blocks=(b0, b0 + 1), threads=1)
+        spent += time.perf_counter() - t0
+        done_bytes += L.k * 128 * L.K // 8 + 2 * L.m * L.k + 2 * L.m * 128 + 2 * L.k + 2 * 128
+        i += 1
+    return {"value": done_bytes / spent / 1e9,
+            "sample": "%d column blocks (one per layer call), %.1f s, fp64 oracle, 1 thread" % (i, spent)}
+
+
+def cpu_oracle_gemm_sample(seconds):
+    """The fp64 oracle on a 64-row slice of the m = 2048 prefill layer
+    (8192 x 28672, K = 3), all host threads, a few 128-column blocks; scaled to
+    the full layer (m / 64 and n / columns done), so the figure is
+    extrapolated."""
+    import oracle
+
+    m, k, n, K = 2048, 8192, 28672, 3
+    L = inputs.make_layer(64, k, n, K, inputs.seed_for(3, 2))
+    threads = oracle.threads_available()
+    cols, spent, b0 = 0, 0.0, 0
+    t_end = time.perf_counter() + seconds
+    while time.perf_counter() < t_end and b0 < n // 128:
+        b1 = min(n // 128, b0 + threads)
+        t0 = time.perf_counter()
+        oracle.linear(L.x, L.trellis, L.suh, L.svh, K, col_blocks=(b0, b1), threads=threads)
+        spent += time.perf_counter() - t0
+        cols += (b1 - b0) * 128
+        b0 = b1
+    flops_done = 2.0 * 64 * k * cols
+    full_s = spent * (m / 64) * (n / cols)
+    return {"value": flops_done / spent / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "extrapolated": True, "full_layer_seconds": full_s,
+            "sample": "64 rows x %d columns of the m=2048 8192x28672 K=3 layer, %.1f s, fp64 oracle with %d "
+                      "OpenMP threads; the full layer scaled by m/64 and n/columns" % (cols, spent, threads)}
+
+
 def make_layers():
     layers = []
     for case, (name, m, k, n, K, outl) in enumerate(workloads.LLAMA8B_DECODE):
@@ -473,7 +519,12 @@ def run_ours(args, rank, world, local_rank):
         if not args.no_cpu_baseline and world == 1:
             cb = cpu_oracle_sample(layers, args.cpu_seconds)
             cb.pop("seconds", None)
+            one = cpu_oracle_one_thread(layers, min(4.0, args.cpu_seconds / 3))
+            cb["value_1_thread"] = one["value"]
+            cb["sample_1_thread"] = one["sample"]
             line["cpu_baseline"] = cb
+            if gemm_info is not None and "tflops" in gemm_info:
+                gemm_info["cpu_baseline"] = cpu_oracle_gemm_sample(min(6.0, args.cpu_seconds / 2))
         print(json.dumps(line), flush=True)
     del graph, graph_ev
     if dist is not None:
