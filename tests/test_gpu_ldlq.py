@@ -78,3 +78,17 @@ def test_ldlq_matches_oracle_bit_exact(k, n, K):
     assert np.array_equal(wh.astype(np.float64), rwhat)
     # and the Hessian-weighted error is the oracle's
     assert OL.proxy_loss(wh, w, h) == pytest.approx(OL.proxy_loss(rwhat, w, h), rel=1e-12)
+
+
+@pytest.mark.parametrize("K", [1, 8])
+def test_ldlq_single_tile_row_is_plain_encoding(K):
+    # k = 16: one block, nothing to feed back, whatever H is (K = 1 also takes
+    # the encoder's global-memory cost vectors)
+    rng = np.random.default_rng(5300 + K)
+    k, n = 16, 48
+    w = rng.standard_normal((k, n)).astype(np.float32)
+    a = rng.standard_normal((k, k))
+    h = a @ a.T + k * np.eye(k)
+    t, _ = _run_ldlq(w, h, K)
+    rt, _ = oracle.encode(w, K)
+    assert np.array_equal(t, rt)
