@@ -86,3 +86,32 @@ def test_gemm_prefill_sampled(case):
     nb = n // 128
     check(layer, y, rows=rows, col_blocks=(0, 1))
     check(layer, y, rows=rows, col_blocks=(nb - 2, nb))
+
+
+# m <= 64: the decoded weights are the MMA's A operand (128 output channels per
+# MMA) and x' its B operand (N = m rounded up to 32).  Shapes with many k
+# blocks per tile split tiles over several CTAs (partial sums and tickets);
+# m = 65 is the first size on the other form.
+@pytest.mark.parametrize("m,k,n,K", [(17, 4096, 2048, 2), (32, 1024, 768, 3), (33, 512, 512, 4),
+                                     (48, 2048, 256, 6), (63, 256, 1024, 8), (64, 4096, 512, 1),
+                                     (2, 8192, 512, 5), (65, 512, 256, 7)])
+def test_gemm_small_m(m, k, n, K):
+    layer = inputs.make_layer(m, k, n, K, seed=6100 + m + K)
+    y, ws = run_gemm(layer)
+    check(layer, y)
+    y2, _ = run_gemm(layer, ws)  # deterministic with the workspace reused
+    assert np.array_equal(y, y2)
+
+
+def test_gemm_small_m_agrees_with_gemv_halves():
+    # m = 32 against two m = 16 GEMV calls on the rows' halves
+    layer = inputs.make_layer(32, 2048, 1024, 3, seed=5)
+    yg, _ = run_gemm(layer)
+    ws = exl3.new_workspace(exl3.exl3_gemv_workspace_size(16, 2048, 1024, 3))
+    for h in range(2):
+        rows = slice(16 * h, 16 * h + 16)
+        yv = exl3.exl3_gemv(dev(layer.x[rows]), dev(layer.trellis), dev(layer.suh), dev(layer.svh), 3,
+                            workspace=ws)
+        yv = yv.cpu().numpy().astype(np.float64)
+        ok, err, bound = within_tolerance(yg[rows], yv)
+        assert ok, (h, err, bound)

@@ -77,25 +77,52 @@ __host__ __device__ constexpr int gemm_trellis_stage_bytes(int K)
     return (kBK / 16) * (kBN / 16) * 32 * K;  // 4 tile rows x 16 tiles
 }
 
-// Trellis ring depth: whatever shared memory the A and B rings leave (up to
-// 227 KB per CTA), at most kMaxTStages stages.
+// Small m (m <= kWaMaxM, one M tile): the decoded weight stage is the A
+// operand instead (M = 128 output channels, MN-major, the same bytes the
+// decoders write for B) and x' the B operand (N = m rounded up to 32,
+// K-major: the first N rows of the x' tile).  Each unit is then two
+// M = 128 x N x 16 MMAs per 16 channels instead of one M = 128 x 256 x 16 of
+// which only m rows are wanted.  The accumulators hold output channels in
+// TMEM lanes and batches in columns, so the epilogue transposes them through
+// a 16 KB shared buffer (32 batches x 128 channels) for the output rotation.
+constexpr int kWaMaxM = 64;
+constexpr int kWaEpiBytes = 32 * 128 * 4;
+
+__host__ __device__ constexpr int gemm_a_stage_bytes(bool wa)
+{
+    return wa ? kWaMaxM * 128 : kAStageBytes;
+}
+
+// Trellis ring depth: whatever shared memory the A and B rings (and the
+// small-m epilogue buffer) leave (up to 227 KB per CTA), at most kMaxTStages
+// stages.
 constexpr int kSmemLimit = 232448;
-constexpr int kTBudget = kSmemLimit - 2048 - kAStages * kAStageBytes - kBStages * kBStageBytes;
 
-__host__ __device__ constexpr int gemm_t_stages(int K)
+__host__ __device__ constexpr int gemm_fixed_bytes(bool wa)
 {
-    return kTBudget / gemm_trellis_stage_bytes(K) > kMaxTStages ? kMaxTStages
-                                                               : kTBudget / gemm_trellis_stage_bytes(K);
+    return 1024 /* alignment slack */ + 1024 /* barriers */ + kAStages * gemm_a_stage_bytes(wa) +
+           kBStages * kBStageBytes + (wa ? kWaEpiBytes : 0);
 }
 
-__host__ __device__ constexpr int gemm_smem_bytes(int K)
+__host__ __device__ constexpr int gemm_t_stages(int K, bool wa)
 {
-    return 1024 /* alignment slack */ + 1024 /* barriers */ + kAStages * kAStageBytes +
-           kBStages * kBStageBytes + gemm_t_stages(K) * gemm_trellis_stage_bytes(K);
+    return (kSmemLimit - gemm_fixed_bytes(wa)) / gemm_trellis_stage_bytes(K) > kMaxTStages
+               ? kMaxTStages
+               : (kSmemLimit - gemm_fixed_bytes(wa)) / gemm_trellis_stage_bytes(K);
 }
 
-static_assert(gemm_t_stages(8) >= 2 && gemm_smem_bytes(8) <= kSmemLimit && gemm_smem_bytes(1) <= kSmemLimit,
+__host__ __device__ constexpr int gemm_smem_bytes(int K, bool wa)
+{
+    return gemm_fixed_bytes(wa) + gemm_t_stages(K, wa) * gemm_trellis_stage_bytes(K);
+}
+
+static_assert(gemm_t_stages(8, false) >= 2 && gemm_smem_bytes(8, false) <= kSmemLimit &&
+                  gemm_smem_bytes(1, false) <= kSmemLimit && gemm_smem_bytes(8, true) <= kSmemLimit &&
+                  gemm_smem_bytes(1, true) <= kSmemLimit,
               "shared memory per CTA");
+static_assert(kWaMaxM % 32 == 0 && kWaMaxM <= kBM && 2 * kWaMaxM * 128 <= kPartialFloats &&
+                  (gemm_a_stage_bytes(true) & 1023) == 0,
+              "small-m tiles");
 
 // ----------------------------------------------------- tcgen05 wrappers ---
 
@@ -208,6 +235,14 @@ __host__ __device__ constexpr uint32_t gemm_idesc()
            ((uint32_t)(kBM >> 4) << 24);
 }
 
+// Small-m form: D f32, A (weights) f16 MN-major, B (x') f16 K-major, M = 128,
+// N = nb.
+__host__ __device__ constexpr uint32_t gemm_idesc_wa(int nb)
+{
+    return (1u << 4) | (0u << 7) | (0u << 10) | (1u << 15) | (0u << 16) | ((uint32_t)(nb >> 3) << 17) |
+           ((uint32_t)(kBM >> 4) << 24);
+}
+
 // 32-point Sylvester Hadamard on 32 fp32 values held by one thread.
 __device__ __forceinline__ void fwht32(float (&v)[32])
 {
@@ -298,6 +333,7 @@ struct GemmParams {
     int kb_count;              // k / 64 units per tile
     uint32_t units;            // tiles * kb_count (units * ctas < 2^32)
     int ctas;                  // grid size G
+    int nb;                    // small-m form: MMA N (m rounded up to 32); 0 otherwise
     uint64_t wait_ns;
     Codebook cb;
 };
@@ -507,18 +543,148 @@ __device__ __forceinline__ bool gemm_epilogue(const GemmParams &p, GemmBars &bar
 }
 
 
-template <int K>
+// Small-m epilogue of one segment [u, se): the accumulators hold output
+// channel tn*256 + 128h + lane in TMEM lane `lane` of half h (columns
+// [h nb, h nb + nb), batch b at column h nb + b).  Partial sums go to the slot
+// as [column][lane] (coalesced over the lanes), the finishing segment sums
+// them in segment order in TMEM, and the output rotation runs per batch row:
+// 32 columns at a time pass through `ebuf` (32 x 128 fp32) so that each warp
+// holds a 128-channel row (4 per lane) for the in-warp Hadamard.
+__device__ __forceinline__ bool gemm_epilogue_wa(const GemmParams &p, GemmBars &bars, uint32_t tmem, float *ebuf,
+                                                 int seg, uint32_t u, uint32_t se, uint32_t U, uint32_t G,
+                                                 uint32_t KB)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int quarter = warp & 3;  // TMEM lanes this warp may access
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const int nrow = quarter * 32 + lane;  // output channel within a 128-channel half
+    const int nb = p.nb;
+    const int nchunks = (2 * nb) >> 5;  // 32-column chunks over both halves
+    volatile int *abort_flag = &bars.abort;
+    const uint32_t t = u / KB;  // one tile row: tile t is column block t
+    const uint32_t tb = t * KB, te = tb + KB;
+    const bool whole = u == tb && se == te;
+    const int tn = (int)t;
+    if (!warp_wait(&bars.acc_full, (uint32_t)seg & 1u, p.wait_ns, 1000)) {
+        if (lane == 0) {
+            record_timeout(p.status);
+            *abort_flag = 1;
+        }
+        return false;
+    }
+    tc_fence_after();
+    if (*abort_flag)
+        return false;
+    int nseg = 1, c_lo = 0;
+    bool finish = true;
+    if (!whole) {
+        c_lo = gemm_owner(tb, U, G);
+        nseg = gemm_owner(te - 1, U, G) - c_lo + 1;
+        float *slot = p.partials + (size_t)gemm_slot(blockIdx.x, tb, U, G) * kPartialFloats;
+#pragma unroll 1
+        for (int cc = 0; cc < nchunks; ++cc) {
+            uint32_t r[32];
+            EXL3_TMEM_LD32(tmem + lane_base + (uint32_t)(32 * cc), r);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                __stcg(slot + (32 * cc + j) * 128 + nrow, __uint_as_float(r[j]));
+        }
+        __threadfence();
+        epi_sync();
+        if (warp == kWarpEpi0 && lane == 0) {
+            const uint32_t prev = atomicAdd(&p.counters[t], 1u);
+            const int last = prev == (uint32_t)(nseg - 1) ? 1 : 0;
+            if (last) {
+                __threadfence();
+                p.counters[t] = 0u;  // every segment has arrived: re-arm for the next call
+            }
+            bars.ticket = last;
+        }
+        epi_sync();
+        finish = bars.ticket != 0;
+    }
+    if (finish && !whole) {
+        // every segment's partials, summed in segment order in TMEM
+#pragma unroll 1
+        for (int j = 0; j < nseg; ++j) {
+            const float *src = p.partials + (size_t)gemm_slot((uint32_t)(c_lo + j), tb, U, G) * kPartialFloats + nrow;
+#pragma unroll 1
+            for (int cc = 0; cc < nchunks; ++cc) {
+                float q[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    q[i] = __ldcg(src + (32 * cc + i) * 128);
+                const uint32_t ta = tmem + lane_base + (uint32_t)(32 * cc);
+                uint32_t r[32];
+                if (j == 0) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        r[i] = __float_as_uint(q[i]);
+                } else {
+                    EXL3_TMEM_LD32(ta, r);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        r[i] = __float_as_uint(__uint_as_float(r[i]) + q[i]);
+                }
+                EXL3_TMEM_ST32(ta, r);
+            }
+            tmem_wait_st();
+        }
+    }
+    if (finish) {
+#pragma unroll 1
+        for (int cc = 0; cc < nchunks; ++cc) {
+            const int h = (32 * cc) / nb, b0 = 32 * cc - h * nb;
+            uint32_t r[32];
+            EXL3_TMEM_LD32(tmem + lane_base + (uint32_t)(32 * cc), r);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                ebuf[j * 128 + nrow] = __uint_as_float(r[j]);
+            epi_sync();
+            const int ncol = tn * kBN + h * 128 + 4 * lane;
+            const uint2 sv2 = *reinterpret_cast<const uint2 *>(p.svh + ncol);
+            const __half2 *sv = reinterpret_cast<const __half2 *>(&sv2);
+#pragma unroll 1
+            for (int i = 0; i < 8; ++i) {
+                const int j = quarter * 8 + i;
+                if (b0 + j < p.m) {
+                    const float4 v4 = *reinterpret_cast<const float4 *>(ebuf + j * 128 + 4 * lane);
+                    float v[4] = {v4.x, v4.y, v4.z, v4.w};
+                    warp_fwht128(v);
+                    const float sc = 0.08838834764831845f;
+                    __half2 o0 = __floats2half2_rn(v[0] * sc * __low2float(sv[0]), v[1] * sc * __high2float(sv[0]));
+                    __half2 o1 = __floats2half2_rn(v[2] * sc * __low2float(sv[1]), v[3] * sc * __high2float(sv[1]));
+                    uint2 out;
+                    out.x = *reinterpret_cast<uint32_t *>(&o0);
+                    out.y = *reinterpret_cast<uint32_t *>(&o1);
+                    *reinterpret_cast<uint2 *>(p.y + (int64_t)(b0 + j) * p.n + ncol) = out;
+                }
+            }
+            epi_sync();  // ebuf is refilled by the next chunk
+        }
+    }
+    // hand the accumulators back to the MMA issuer
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0)
+        mbar_arrive(&bars.acc_empty);
+    return true;
+}
+
+template <int K, bool WA>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmParams p)
 {
-    constexpr int TS = gemm_t_stages(K);
+    constexpr int TS = gemm_t_stages(K, WA);
     constexpr int kTrBytes = gemm_trellis_stage_bytes(K);
     constexpr int kTileRowBytes = (kBN / 16) * 32 * K;
+    constexpr int AS = gemm_a_stage_bytes(WA);
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
     GemmBars &bars = *reinterpret_cast<GemmBars *>(smem);
     unsigned char *aring = smem + 1024;
-    unsigned char *bring = aring + kAStages * kAStageBytes;
-    unsigned char *tring = bring + kBStages * kBStageBytes;
+    unsigned char *bring = aring + kAStages * AS;
+    float *ebuf = reinterpret_cast<float *>(bring + kBStages * kBStageBytes);  // small-m epilogue only
+    unsigned char *tring = bring + kBStages * kBStageBytes + (WA ? kWaEpiBytes : 0);
     volatile int *abort_flag = &bars.abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -574,11 +740,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmParams 
                     *abort_flag = 1;
                     break;
                 }
-                unsigned char *dst = aring + s * kAStageBytes;
-                mbar_arrive_expect_tx(&bars.afull[s], (uint32_t)(mt_count * kATileBytes));
-                for (int mt = 0; mt < mt_count; ++mt) {
-                    const int64_t tile = (int64_t)(tm * kMT + mt) * (p.k / kBK) + kb;
-                    bulk_g2s(dst + mt * kATileBytes, p.xt + tile * kATileBytes, kATileBytes, &bars.afull[s]);
+                unsigned char *dst = aring + s * AS;
+                if constexpr (WA) {
+                    // the first nb rows (batches) of x' tile (0, kb): nb x 128 contiguous bytes
+                    mbar_arrive_expect_tx(&bars.afull[s], (uint32_t)(p.nb * 128));
+                    bulk_g2s(dst, p.xt + (int64_t)kb * kATileBytes, (uint32_t)(p.nb * 128), &bars.afull[s]);
+                } else {
+                    mbar_arrive_expect_tx(&bars.afull[s], (uint32_t)(mt_count * kATileBytes));
+                    for (int mt = 0; mt < mt_count; ++mt) {
+                        const int64_t tile = (int64_t)(tm * kMT + mt) * (p.k / kBK) + kb;
+                        bulk_g2s(dst + mt * kATileBytes, p.xt + tile * kATileBytes, kATileBytes, &bars.afull[s]);
+                    }
                 }
                 issued = i + 1;
                 if (++kb == (int)KB) {
@@ -627,7 +799,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmParams 
     } else if (warp == kWarpMma) {
         // ----------------------------------------------------- MMA issuer ---
         if (lane == 0) {
-            const uint32_t idesc = gemm_idesc();
+            const uint32_t idesc = WA ? gemm_idesc_wa(p.nb) : gemm_idesc();
             uint32_t t = u0 / KB;
             int kb = (int)(u0 - t * KB);
             int mt_count = (p.m - (int)(t / p.tiles_n) * kBM * kMT) > kBM ? kMT : 1;
@@ -651,15 +823,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmParams 
                     break;
                 }
                 tc_fence_after();
-                const uint32_t a0 = smem_addr(aring + sa * kAStageBytes);
+                const uint32_t a0 = smem_addr(aring + sa * AS);
                 const uint32_t b0 = smem_addr(bring + sb * kBStageBytes);
+                if constexpr (WA) {
+                    // weights (the decoded stage, MN-major: 64-channel groups at
+                    // 8192 B, 8-row k atoms at 1024 B) as A, one MMA per
+                    // 128-channel half h into TMEM columns [h nb, h nb + nb)
 #pragma unroll
-                for (int kk = 0; kk < kBK / 16; ++kk) {
-                    const uint64_t bdesc = smem_desc(b0 + kk * 2048, 8192, 1024);
-                    for (int mt = 0; mt < mt_count; ++mt) {
-                        const uint64_t adesc = smem_desc(a0 + mt * kATileBytes + kk * 32, 16, 1024);
-                        mma_f16_ss(tmem + (uint32_t)(mt * kBN), adesc, bdesc, idesc,
-                                   (!seg_start || kk) ? 1u : 0u);
+                    for (int kk = 0; kk < kBK / 16; ++kk) {
+                        const uint64_t xdesc = smem_desc(a0 + kk * 32, 16, 1024);
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const uint64_t wdesc = smem_desc(b0 + h * 16384 + kk * 2048, 8192, 1024);
+                            mma_f16_ss(tmem + (uint32_t)(h * p.nb), wdesc, xdesc, idesc,
+                                       (!seg_start || kk) ? 1u : 0u);
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk) {
+                        const uint64_t bdesc = smem_desc(b0 + kk * 2048, 8192, 1024);
+                        for (int mt = 0; mt < mt_count; ++mt) {
+                            const uint64_t adesc = smem_desc(a0 + mt * kATileBytes + kk * 32, 16, 1024);
+                            mma_f16_ss(tmem + (uint32_t)(mt * kBN), adesc, bdesc, idesc,
+                                       (!seg_start || kk) ? 1u : 0u);
+                        }
                     }
                 }
                 mma_commit(&bars.aempty[sa]);
@@ -689,7 +877,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmParams 
         for (int seg = 0; seg_u < u1; ++seg) {
             const uint32_t te = (seg_u / KB + 1) * KB;
             const uint32_t seg_e = te < u1 ? te : u1;
-            if (!gemm_epilogue(p, bars, tmem, seg, seg_u, seg_e, U, G, KB))
+            const bool ok = WA ? gemm_epilogue_wa(p, bars, tmem, ebuf, seg, seg_u, seg_e, U, G, KB)
+                               : gemm_epilogue(p, bars, tmem, seg, seg_u, seg_e, U, G, KB);
+            if (!ok)
                 break;
             seg_u = seg_e;
         }
@@ -762,11 +952,11 @@ static GemmPlan gemm_plan(int64_t m, int64_t k, int64_t n, int sms)
     return pl;
 }
 
-template <int K>
+template <int K, bool WA>
 static exl3_status launch_gemm_t(const GemmParams &p, cudaStream_t stream)
 {
-    constexpr int smem = gemm_smem_bytes(K);
-    auto kern = gemm_kernel<K>;
+    constexpr int smem = gemm_smem_bytes(K, WA);
+    auto kern = gemm_kernel<K, WA>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return EXL3_ERR_CUDA;
     if (launch_kernel(kern, dim3(p.ctas), dim3(kGemmThreads), (size_t)smem, stream, p) != cudaSuccess)
@@ -825,14 +1015,28 @@ extern "C" exl3_status exl3_gemm(const void *x, const uint16_t *trellis, const v
     p.ctas = pl.ctas;
     p.wait_ns = wait_limit_ns();
     p.cb = codebook_constants();
+    const bool wa = m <= kWaMaxM;
+    p.nb = wa ? (int)((m + 31) & ~(int64_t)31) : 0;
+    if (wa) {
+        switch (K) {
+        case 1: return launch_gemm_t<1, true>(p, s);
+        case 2: return launch_gemm_t<2, true>(p, s);
+        case 3: return launch_gemm_t<3, true>(p, s);
+        case 4: return launch_gemm_t<4, true>(p, s);
+        case 5: return launch_gemm_t<5, true>(p, s);
+        case 6: return launch_gemm_t<6, true>(p, s);
+        case 7: return launch_gemm_t<7, true>(p, s);
+        default: return launch_gemm_t<8, true>(p, s);
+        }
+    }
     switch (K) {
-    case 1: return launch_gemm_t<1>(p, s);
-    case 2: return launch_gemm_t<2>(p, s);
-    case 3: return launch_gemm_t<3>(p, s);
-    case 4: return launch_gemm_t<4>(p, s);
-    case 5: return launch_gemm_t<5>(p, s);
-    case 6: return launch_gemm_t<6>(p, s);
-    case 7: return launch_gemm_t<7>(p, s);
-    default: return launch_gemm_t<8>(p, s);
+    case 1: return launch_gemm_t<1, false>(p, s);
+    case 2: return launch_gemm_t<2, false>(p, s);
+    case 3: return launch_gemm_t<3, false>(p, s);
+    case 4: return launch_gemm_t<4, false>(p, s);
+    case 5: return launch_gemm_t<5, false>(p, s);
+    case 6: return launch_gemm_t<6, false>(p, s);
+    case 7: return launch_gemm_t<7, false>(p, s);
+    default: return launch_gemm_t<8, false>(p, s);
     }
 }
