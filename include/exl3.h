@@ -186,7 +186,10 @@ exl3_status exl3_gemv_noalloc(const void *x, const uint16_t *trellis, const void
  * is persistent (one CTA per SM) and splits the work evenly over the CTAs by
  * (256 x 256 output tile, 64-channel k block) units, so a tile can be shared
  * by several CTAs; their fp32 partial sums meet in the workspace and are
- * added in a fixed order, so results are deterministic.
+ * added in a fixed order, so results are deterministic.  For m <= 64 the
+ * decoded weights are the MMA's A operand (128 output channels per MMA) and
+ * the rotated activations its B operand (N = m rounded up to 32), so a small
+ * batch does not pay for 128-row MMAs; the result is the same function.
  * `workspace` (at least exl3_gemm_workspace_size bytes -- a size that depends
  * on the current device's SM count, so query it on the device that runs the
  * call -- zero-filled once after allocation) holds a status word, per-tile
