@@ -41,6 +41,12 @@
 //                 H4 (x) H32 (32-point butterflies in registers, a TMEM round
 //                 trip, then the 4-point stage), svh/sqrt(128), fp16 y; or the
 //                 partial-sum write and the ticket.
+//   For m <= 64 the same kernel runs with the operands swapped (template
+//   flag WA): the decoded stage is the A operand (M = 128 output channels per
+//   MMA, two per 16-channel step), x' rows 0 .. N-1 the B operand (N = m
+//   rounded up to 32), and the epilogue transposes the accumulators (channels
+//   in TMEM lanes, batches in columns) through shared memory for the output
+//   rotation.
 //   Shared memory is addressed from the dynamic shared array (the 1024-byte
 //   alignment the swizzled tiles need is an offset, not an integer cast), so
 //   the decoders' loads and stores stay shared-space instructions.
