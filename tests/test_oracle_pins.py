@@ -78,6 +78,31 @@ def test_codebook_whole_table_invariants(table):
     assert (wd ** 2).sum() == pytest.approx(float(g["sum_sq"]), rel=1e-15)
 
 
+def test_codebook_split_sum_bound(table):
+    # The word's two halves, from the definition with numpy (not the oracle's
+    # code): their exact sum rounds (nearest even) to the oracle's value, the
+    # count of states where that rounding changes anything is the golden one,
+    # and the change is at most half an fp16 ulp, i.e. at most 2^-11 relative
+    # -- the bound behind computing x * (hi + lo) exactly instead of with the
+    # rounded weight.
+    g = {row[0]: row[1] for row in read_golden("codebook_stats.txt")}
+    s = np.arange(65536, dtype=np.uint64)
+    v = (s * 89226354 + 64248484) & 0xffffffff
+    v = (v & 0x8fff8fff) ^ 0x3b603b60
+    hi = (v >> 16).astype(np.uint16).view(np.float16).astype(np.float64)
+    lo = (v & 0xffff).astype(np.uint16).view(np.float16).astype(np.float64)
+    exact = hi + lo  # exact in fp64: both halves are fp16 with exponents -3..0
+    w = table.view(np.float16).astype(np.float64)
+    assert np.array_equal(exact.astype(np.float16).view(np.uint16), table)
+    d = np.abs(exact - w)
+    assert int((d > 0).sum()) == int(g["rounded_sums"])
+    nz = w != 0
+    ulp = 2.0 ** (np.floor(np.log2(np.abs(w[nz]))) - 10)
+    assert (d[nz] <= 0.5 * ulp).all()
+    assert (d[nz] / np.abs(w[nz])).max() == 2.0 ** -11
+    assert (d[~nz] == 0).all()
+
+
 def test_codebook_halves_range(table):
     # |w| < 4 since each half is in +-[0.125, 2); and w never subnormal
     wd = table.view(np.float16).astype(np.float64)
