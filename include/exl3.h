@@ -163,11 +163,15 @@ exl3_status exl3_gemv_multi(const exl3_linear *layers, int count, int64_t m, voi
  *   - Shapes whose scratch exceeds that maximum are rejected with
  *     EXL3_ERR_WORKSPACE before anything is launched (exl3_gemv_workspace_size
  *     tells how much a shape needs).
- *   - The first call on a device looks the array's device address up
- *     (cudaGetSymbolAddress) and caches it; make that first call before any
- *     stream capture on that device.
+ *   - The array's device address is looked up (cudaGetSymbolAddress) on the
+ *     first call on a device and again whenever the current context changes
+ *     (after cudaDeviceReset, for example).  The lookup cannot run inside a
+ *     stream capture: a call that needs it while `stream` is capturing
+ *     returns EXL3_ERR_UNSUPPORTED, so make the first call on a device
+ *     outside any capture.
  *   - Every call on a device shares the one array and it keeps the last call's
- *     contents: each call first clears the arrival counters on its stream, and
+ *     contents: each call first clears the status word and the arrival
+ *     counters on its stream (one cudaMemsetAsync, which allocates nothing), and
  *     calls that can overlap on the GPU (different streams, or concurrent
  *     host threads) race on the array and must not be issued.
  *   - No cudaMalloc, cudaFree or other allocating routine is called.

@@ -194,3 +194,29 @@ def test_udu_and_ldlq_argument_errors_and_sizes():
     need = lib.exl3_ldlq_workspace_size(64, 128, 4)
     assert need >= 64 * 64 * 8 + 64 * 128 * 8 + lib.exl3_encode_workspace_size(16, 128, 4)
     assert lib.exl3_ldlq_workspace_size(64, 40, 4) == 0
+
+
+def test_binding_checks_tensor_sizes_before_the_call():
+    # the binding compares every tensor with (m, k, n, K) before anything
+    # reaches the C ABI (CPU tensors suffice: the check comes first)
+    import torch
+    m, k, n, K = 2, 256, 128, 3
+    x = torch.zeros((m, k), dtype=torch.float16)
+    t = torch.zeros((k // 16, n // 16, 16 * K), dtype=torch.uint16)
+    suh = torch.ones(k, dtype=torch.float16)
+    svh = torch.ones(n, dtype=torch.float16)
+    y = torch.empty((m, n), dtype=torch.float16)
+    bad = [
+        dict(trellis=t[:-1]),
+        dict(suh=suh[:-1]),
+        dict(y=torch.empty((m, n - 1), dtype=torch.float16)),
+        dict(K=K + 1),
+    ]
+    for change in bad:
+        a = dict(x=x, trellis=t, suh=suh, svh=svh, K=K, y=y)
+        a.update(change)
+        for fn in (exl3.exl3_gemv, exl3.exl3_gemm):
+            with pytest.raises(ValueError):
+                fn(a["x"], a["trellis"], a["suh"], a["svh"], a["K"], y=a["y"], workspace=torch.zeros(256, dtype=torch.uint8))
+        with pytest.raises(ValueError):
+            exl3.exl3_gemv_noalloc(a["x"], a["trellis"], a["suh"], a["svh"], a["K"], y=a["y"])

@@ -8,12 +8,15 @@ library.  These tests call it through the C ABI and check that it gives the
 same outputs as exl3_gemv, within the stated output tolerance, on two calls in
 a row (the array keeps the previous call's contents, so the second call
 checks that nothing stale leaks through).  The file is named to be collected
-last; it passes alone in a fresh process as well.
+last; it passes alone in a fresh process as well.  The outputs are also
+checked against the fp64 oracle, so that a fault shared by both entry points
+(the scratch layout, say) cannot pass unseen.
 """
 import numpy as np
 import pytest
 import torch
 
+import oracle
 from conftest import within_tolerance
 from trellis_coded_bit_b200 import exl3, inputs
 
@@ -49,6 +52,28 @@ def test_noalloc_matches_gemv_on_two_calls_in_a_row(m, k, n, K):
             got = y.cpu().numpy().astype(np.float64)
             ok, err, bound = within_tolerance(got, ref)
             assert ok, "max err %.4g > bound %.4g" % (err, bound)
+        # against the oracle, on the first, a middle and the last column block
+        nb = n // 128
+        for cb in sorted({0, nb // 2, nb - 1}):
+            want = oracle.linear(L.x, L.trellis, L.suh, L.svh, K, col_blocks=(cb, cb + 1))
+            got = y2.cpu().numpy().astype(np.float64)[:, cb * 128:(cb + 1) * 128]
+            ok, err, bound = within_tolerance(got, want)
+            assert ok, "block %d: max err %.4g > bound %.4g" % (cb, err, bound)
+
+
+def test_noalloc_split_k_shape_matches_the_oracle():
+    # k = 8192 with 256 column blocks: more CTAs than column blocks, so every
+    # block is split over several CTAs whose partials meet in the scratch array
+    m, k, n, K = 2, 8192, 2048, 3
+    assert exl3.exl3_gemv_workspace_size(m, k, n, K) <= exl3.exl3_gemv_noalloc_max_scratch()
+    L = inputs.make_layer(m, k, n, K, seed=930)
+    y = torch.empty((m, n), dtype=torch.float16, device="cuda")
+    exl3.exl3_gemv_noalloc(dev(L.x), dev(L.trellis), dev(L.suh), dev(L.svh), K, y=y)
+    got = y.cpu().numpy().astype(np.float64)
+    for cb in (0, 7, 15):
+        want = oracle.linear(L.x, L.trellis, L.suh, L.svh, K, col_blocks=(cb, cb + 1))
+        ok, err, bound = within_tolerance(got[:, cb * 128:(cb + 1) * 128], want)
+        assert ok, "block %d: max err %.4g > bound %.4g" % (cb, err, bound)
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():

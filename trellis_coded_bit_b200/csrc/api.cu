@@ -24,6 +24,32 @@ uint64_t wait_limit_ns()
     return g_wait_ns.load(std::memory_order_relaxed);
 }
 
+// SM count of the current device, looked up once per device (a read-only
+// property of the hardware, so the cache never goes stale).
+int num_sms()
+{
+    constexpr int kDevs = 64;
+    static std::atomic<int> cache[kDevs];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return 148;
+    }
+    if (dev >= 0 && dev < kDevs) {
+        const int v = cache[dev].load(std::memory_order_relaxed);
+        if (v > 0)
+            return v;
+    }
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) {
+        cudaGetLastError();
+        v = 148;
+    }
+    if (dev >= 0 && dev < kDevs)
+        cache[dev].store(v, std::memory_order_relaxed);
+    return v;
+}
+
 }  // namespace exl3
 
 extern "C" const char *exl3_status_string(int status)

@@ -34,7 +34,11 @@
 //   * Lane (g, t) owns tile g of the 128-column block and, in k-step ks, the
 //     two adjacent tile rows 8ks + 2t and 8ks + 2t + 1: one contiguous run of
 //     2K + 1 words (with the prefix word) whose 32 bit windows are
-//     compile-time byte permutes (pair_states).  Weight (row 8ks + 2t + p,
+//     compile-time byte permutes and multiplies (pair_codes), which move what
+//     they can from the ALU pipe (byte permutes and the codebook's mask/xor)
+//     to the FMA pipe (the codebook's multiply, shifts as multiplies, and an
+//     exact correction that lets a window skip its zero-fill when the 16 bits
+//     above it are another window's state).  Weight (row 8ks + 2t + p,
 //     column c) goes to A row g + 8(c & 1), k-pair t + 4p of MMA c / 2, so
 //     MMA j accumulates columns 2j and 2j + 1 of every tile of the block.
 //   * Each warp streams its units through its own 3-deep cp.async ring in
@@ -62,6 +66,12 @@ constexpr int kGemvThreads = 32 * kGemvWarps;
 // entries of absent batches are zero (they feed only B columns whose
 // accumulators are never stored).
 constexpr int kGemvActBlock = 512;
+
+// The first bytes of every GEMV workspace hold the words a call needs to find
+// at zero when it starts (status word, arrival counters; every call leaves
+// them at zero), and no call writes data there, so one workspace can serve
+// calls of any shapes in turn.
+constexpr size_t kGemvSyncArea = 64 * 1024;
 
 __host__ __device__ inline int gemv_mg(int64_t m)
 {
@@ -217,42 +227,90 @@ __device__ __forceinline__ void cp_async_wait()
     asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
-// The 32 states of a row pair from its run of words.  R[0] holds the prefix
-// word in its upper half, R[i] (i = 1..K) holds the pair's words 2i - 2
-// (lower half) and 2i - 1 (upper half).  Counting stream positions from the
-// prefix word W'[0] (W'[i] = positions 16i .. 16i + 15; W'[2i-1] is R[i]'s
-// lower half, W'[2i] its upper half), weight jj (row jj / 16, column jj % 16)
-// has the window ending at position e = 16 + (jj + 1) K.  When e is a
-// multiple of 16 the window is the word W'[e/16 - 1]; otherwise it lies in
-// V = W'[a-1]:W'[a] (a = e / 16, as one big-endian 32-bit value) shifted
-// right by c = 16 - e % 16, and is one byte permute with zero fill of V or of
-// V times 2^(8 - c % 8) (a left shift, as a multiply on the FMA pipe).  All
-// selectors are compile-time constants, and the V values and their shifted
-// copies are shared between windows.
+// The 32 codebook words of a row pair from its run of words.  R[0] holds the
+// prefix word in its upper half, R[i] (i = 1..K) holds the pair's words
+// 2i - 2 (lower half) and 2i - 1 (upper half).  Counting stream positions
+// from the prefix word W'[0] (W'[i] = positions 16i .. 16i + 15; W'[2i-1] is
+// R[i]'s lower half, W'[2i] its upper half), weight jj (row jj / 16, column
+// jj % 16) has the window ending at position e = 16 + (jj + 1) K.
+//   * When e is a multiple of 16 the window is the word W'[e/16 - 1]: an
+//     upper half is one byte permute with zero fill; a lower half, when K
+//     divides 16, needs no extraction at all: with R = W'[w+1] 2^16 + W'[w]
+//     and W'[w+1] itself the state of weight jj' = jj + 16/K, R*C1 + C2
+//     differs from the wanted s*C1 + C2 only by (W'[w+1] C1 mod 2^16) 2^16,
+//     and W'[w+1] C1 mod 2^16 is the low half of jj''s own product less C2:
+//     so v = R*C1 + (C2 + C2 2^16) - v' 2^16, two multiply-adds on the FMA
+//     pipe, exact mod 2^32.
+//   * A window 8 bits off a word boundary that lies inside one loaded
+//     register (a even) is one byte permute of that register.  For K = 8 one
+//     that straddles two registers is the low half of the 32-bit window
+//     ending at the same place (one byte permute of the two registers),
+//     whose upper half is the state of weight jj - 2, and is corrected the
+//     same way.
+//   * Otherwise the window lies in V = W'[a-1]:W'[a] (a = e / 16, as one
+//     big-endian 32-bit value) shifted right by c = 16 - e % 16, and is one
+//     byte permute with zero fill of V, or of V times 2^(8 - c % 8) (a left
+//     shift, as a multiply on the FMA pipe).
+// All selectors are compile-time constants, and the V values and their
+// shifted copies are shared between windows.  The result is the codebook
+// word (v & mask) ^ xor of each window's state.
 template <int K>
-__device__ __forceinline__ void pair_states(const uint32_t (&R)[K + 1], uint32_t (&s)[32], const GemvMults &mu)
+__device__ __forceinline__ void pair_codes(const uint32_t (&R)[K + 1], uint32_t (&w)[32], const Codebook &cb,
+                                           uint32_t c2p, const GemvMults &mu)
 {
+    constexpr bool kJunk = (16 % K) == 0;
+    constexpr int kStep = kJunk ? 16 / K : 0;
+    uint32_t v[32];
 #pragma unroll
     for (int jj = 0; jj < 32; ++jj) {
         const int e = 16 + (jj + 1) * K;
         const int a = e >> 4, rb = e & 15;
+        const int c = 16 - rb;
+        uint32_t s;
         if (rb == 0) {
-            const int w = a - 1;
-            s[jj] = (w & 1) ? __byte_perm(R[(w + 1) >> 1], 0u, 0x4410u) : __byte_perm(R[w >> 1], 0u, 0x4432u);
-        } else {
-            const uint32_t v = (a & 1) ? __byte_perm(R[(a - 1) >> 1], R[(a + 1) >> 1], 0x3254u)
-                                       : __byte_perm(R[a >> 1], 0u, 0x1032u);
-            const int c = 16 - rb, r = c & 7, cb = c >> 3;
-            if (r == 0) {
-                s[jj] = __byte_perm(v, 0u, 0x4400u | ((uint32_t)(cb + 1) << 4) | (uint32_t)cb);
+            const int wd = a - 1;
+            if (wd & 1) {
+                if (kJunk)
+                    continue;  // corrected below from the window 16 bits later
+                s = __byte_perm(R[(wd + 1) >> 1], 0u, 0x4410u);
             } else {
-                // bits [c, c + 16) of v are bits [8(cb + 1), 8(cb + 1) + 16) of
-                // v * 2^(8 - r); the bits shifted out lie above the window
-                const uint32_t vs = v * mu.pow2[8 - r];
-                s[jj] = __byte_perm(vs, 0u, 0x4400u | ((uint32_t)(cb + 2) << 4) | (uint32_t)(cb + 1));
+                s = __byte_perm(R[wd >> 1], 0u, 0x4432u);
+            }
+        } else if (c == 8 && !(a & 1)) {
+            s = __byte_perm(R[a >> 1], 0u, 0x4403u);
+        } else if (c == 8 && K == 8 && jj >= kStep) {
+            continue;  // corrected below from the window 16 bits earlier
+        } else {
+            const uint32_t vv = (a & 1) ? __byte_perm(R[(a - 1) >> 1], R[(a + 1) >> 1], 0x3254u)
+                                        : __byte_perm(R[a >> 1], 0u, 0x1032u);
+            const int r = c & 7, cbt = c >> 3;
+            if (r == 0) {
+                s = __byte_perm(vv, 0u, 0x4400u | ((uint32_t)(cbt + 1) << 4) | (uint32_t)cbt);
+            } else {
+                // bits [c, c + 16) of vv are bits [8(cbt + 1), 8(cbt + 1) + 16) of
+                // vv * 2^(8 - r); the bits shifted out lie above the window
+                const uint32_t vs = vv * mu.pow2[8 - r];
+                s = __byte_perm(vs, 0u, 0x4400u | ((uint32_t)(cbt + 2) << 4) | (uint32_t)(cbt + 1));
+            }
+        }
+        v[jj] = s * cb.mul + cb.add;
+    }
+    if constexpr (kJunk) {
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+            const int e = 16 + (jj + 1) * K;
+            const int a = e >> 4, rb = e & 15;
+            if (rb == 0 && ((a - 1) & 1)) {
+                v[jj] = v[jj + kStep] * 0xFFFF0000u + (R[a >> 1] * cb.mul + c2p);
+            } else if (K == 8 && rb == 8 && (a & 1) && jj >= kStep) {
+                const uint32_t xw = __byte_perm(R[(a - 1) >> 1], R[(a + 1) >> 1], 0x0325u);
+                v[jj] = v[jj - kStep] * 0xFFFF0000u + (xw * cb.mul + c2p);
             }
         }
     }
+#pragma unroll
+    for (int jj = 0; jj < 32; ++jj)
+        w[jj] = (v[jj] & cb.mask) ^ cb.xr;
 }
 
 // The lane's pointers into a stage of its ring (stage 0 as set up; the loop
@@ -319,12 +377,11 @@ __device__ __forceinline__ void mac_unit(const GemvLanePtrs &lp, const Codebook 
             load_pair<K, 0>(lp, R);
         else
             load_pair<K, 1>(lp, R);
-        uint32_t st[32];
-        pair_states<K>(R, st, mu);
+        uint32_t wv[32];
+        pair_codes<K>(R, wv, cb, cb.add + (cb.add << 16), mu);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            const uint32_t a[4] = {codebook_word(st[2 * j], cb), codebook_word(st[2 * j + 1], cb),
-                                   codebook_word(st[16 + 2 * j], cb), codebook_word(st[17 + 2 * j], cb)};
+            const uint32_t a[4] = {wv[2 * j], wv[2 * j + 1], wv[16 + 2 * j], wv[17 + 2 * j]};
 #pragma unroll
             for (int mg = 0; mg < MG; ++mg)
                 mma_16816(acc[mg][j], a, B[mg][0], B[mg][1]);
@@ -598,15 +655,15 @@ __device__ __forceinline__ void gemv_cta(const GemvParams &p, const GemvGroup &g
             float *part = SL.partials + ((int64_t)cbk * SL.max_seg) * m * 128;
             for (int e = tid; e < m * 128; e += kGemvThreads)
                 part[(int64_t)j * m * 128 + e] = red[e];
-            __threadfence();
             __syncthreads();
             if (tid == 0) {
+                __threadfence();  // the barrier orders the other threads' stores before this fence
                 const uint32_t ticket = atomicAdd(&SL.counters[cbk], 1u);
                 *flag = (ticket == (uint32_t)(nseg - 1)) ? 1 : 0;
+                __threadfence();
             }
             __syncthreads();
             if (*flag == 1) {
-                __threadfence();
                 // segment order, eight independent loads in flight per thread
                 for (int e = tid; e < m * 128; e += kGemvThreads) {
                     float a8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -654,28 +711,11 @@ __global__ void __launch_bounds__(kGemvThreads, MG == 1 ? 2 : 1) gemv_kernel(con
 
 // ------------------------------------------------------------- dispatch ---
 
-static int g_num_sms = 0;
-
-int num_sms()
-{
-    if (g_num_sms <= 0) {
-        int dev = 0;
-        int v = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) {
-            cudaGetLastError();
-            v = 148;
-        }
-        g_num_sms = v;
-    }
-    return g_num_sms;
-}
-
 // Plan of one launch over `count` layers (same m): the K groups and their
 // CTAs, shared memory, and the workspace layout -- [0, 256) status word; the
-// layers' arrival counters (one per column block, consecutive); then per
-// layer its activation blocks (k / 16 * MG * 512 bytes) and split partials
-// [n/128][max_seg][m][128].  Workspace offsets are indexed by the layer's
+// layers' arrival counters (one per column block, consecutive); from
+// kGemvSyncArea on, per layer its activation blocks (k / 16 * MG * 512 bytes)
+// and split partials [n/128][max_seg][m][128].  Workspace offsets are indexed by the layer's
 // place in the call; the group order is `order`.
 struct GemvPlan {
     int ctas, smem, ngroups;
@@ -683,7 +723,8 @@ struct GemvPlan {
     int order[kGemvMaxLayers];  // call index of the plan's l-th layer (grouped by K)
     int64_t unit_begin[kGemvMaxLayers];
     int cb_begin[kGemvMaxLayers], max_seg[kGemvMaxLayers];  // by plan index
-    size_t counters[kGemvMaxLayers], acts[kGemvMaxLayers], partials[kGemvMaxLayers], total;  // by call index
+    size_t counters[kGemvMaxLayers], acts[kGemvMaxLayers], partials[kGemvMaxLayers];  // by call index
+    size_t sync_bytes, total;
 };
 
 // Relative time of one unit at m = 1 by K: each K group of the Llama-3.1-8B
@@ -803,6 +844,8 @@ static GemvPlan gemv_plan(const int64_t *k, const int64_t *n, const int *K, int 
         off += (size_t)(n[l] / 128) * 4;
     }
     off = (off + 255) / 256 * 256;
+    pl.sync_bytes = off;
+    off = off > kGemvSyncArea ? off : kGemvSyncArea;
     for (int q = 0; q < pl.ngroups; ++q) {
         const GemvGroup &gr = pl.grp[q];
         for (int i = gr.l_begin; i < gr.l_end; ++i) {
@@ -829,6 +872,13 @@ static GemvPlan gemv_plan(const int64_t *k, const int64_t *n, const int *K, int 
     }
     pl.total = off;
     return pl;
+}
+
+// Bytes at the start of a one-layer workspace that must be zero when a call
+// starts (status word and arrival counters).
+size_t gemv_sync_bytes(int64_t m, int64_t k, int64_t n, int K, int sms)
+{
+    return gemv_plan(&k, &n, &K, 1, m, sms).sync_bytes;
 }
 
 size_t gemv_workspace_bytes(int64_t m, int64_t k, int64_t n, int sms)
@@ -1040,12 +1090,13 @@ extern "C" exl3_status exl3_gemv_multi(const exl3_linear *layers, int count, int
 // ------------------------------------------------ no-allocation variant ---
 //
 // exl3_gemv_noalloc runs the GEMV above with its scratch (split-k partials
-// and arrival counters) in a fixed array compiled into the library, for
-// callers that must not allocate device memory themselves.  The array is a
-// file-scope __device__ symbol: every GPU that loads the library holds its
-// kNoAllocScratchBytes until the process exits.  In host code the symbol's
-// name is only a host-side stand-in, so the device address is looked up once
-// per device with cudaGetSymbolAddress (with that device current) and cached.
+// and arrival counters) in a fixed array
+// compiled into the library, for callers that must not allocate device
+// memory themselves.  The array is a file-scope __device__ symbol: every GPU
+// that loads the library holds its kNoAllocScratchBytes until the process
+// exits.  In host code the symbol's name is only a host-side stand-in, so the
+// device address is looked up with cudaGetSymbolAddress (with the device
+// current) and cached per device and context.
 
 #include <mutex>
 
@@ -1056,25 +1107,60 @@ constexpr size_t kNoAllocScratchBytes = 4u << 20;  // 4 MiB per device
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
-static void *g_noalloc_ptr[kMaxDevices];
+struct NoAllocCache {
+    void *ptr;
+    void *ctx;  // the context (CUcontext) the address belongs to
+};
+static NoAllocCache g_noalloc[kMaxDevices];
 static std::mutex g_noalloc_mutex;
 
-// Device address of this device's scratch array (set up on first use).
-static exl3_status noalloc_scratch(void **out)
+// The driver's cuCtxGetCurrent, fetched through the runtime (the library
+// links only the runtime).  Returns null when it is unavailable.
+static void *current_context()
+{
+    typedef int (*GetCurrent)(void **);
+    static GetCurrent fn = []() -> GetCurrent {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<GetCurrent>(f);
+    }();
+    void *ctx = nullptr;
+    if (!fn || fn(&ctx) != 0)
+        return nullptr;
+    return ctx;
+}
+
+// Device address of this device's scratch array.  It is looked up again
+// whenever the current context differs from the one it was looked up in (a
+// cudaDeviceReset makes a new primary context, and the old address with it
+// invalid).  Inside a stream capture the lookup is refused with
+// EXL3_ERR_UNSUPPORTED: make a first call on the device outside capture.
+static exl3_status noalloc_scratch(cudaStream_t stream, void **out)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess)
         return EXL3_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices)
         return EXL3_ERR_UNSUPPORTED;
+    void *ctx = current_context();
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_ptr[dev]) {
+    if (!g_noalloc[dev].ptr || g_noalloc[dev].ctx != ctx) {
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess)
+            return EXL3_ERR_CUDA;
+        if (cs != cudaStreamCaptureStatusNone)
+            return EXL3_ERR_UNSUPPORTED;
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)
             return EXL3_ERR_CUDA;
-        g_noalloc_ptr[dev] = p;
+        ctx = current_context();
+        g_noalloc[dev].ptr = p;
+        g_noalloc[dev].ctx = ctx;
     }
-    *out = g_noalloc_ptr[dev];
+    *out = g_noalloc[dev].ptr;
     return EXL3_OK;
 }
 
@@ -1099,14 +1185,14 @@ extern "C" exl3_status exl3_gemv_noalloc(const void *x, const uint16_t *trellis,
     if (need > kNoAllocScratchBytes)
         return EXL3_ERR_WORKSPACE;  // this shape needs more scratch than the built-in array
     void *scratch = nullptr;
-    const exl3_status sst = noalloc_scratch(&scratch);
+    const exl3_status sst = noalloc_scratch((cudaStream_t)stream, &scratch);
     if (sst != EXL3_OK)
         return sst;
-    // the array keeps whatever the last call left: the arrival counters must
-    // start at zero (the kernel re-arms them, but a call that never finished
-    // could have left them set), so clear them on the caller's stream
-    const size_t counter_bytes = 256 + (size_t)((n / 128) * 4 + 255) / 256 * 256;
-    if (cudaMemsetAsync(scratch, 0, counter_bytes, (cudaStream_t)stream) != cudaSuccess)
+    // the array keeps whatever the last call left: the status word and the
+    // arrival counters must start at zero (the kernel re-arms the counters,
+    // but a call that never finished could have left them set), so clear
+    // them on the caller's stream
+    if (cudaMemsetAsync(scratch, 0, gemv_sync_bytes(m, k, n, K, num_sms()), (cudaStream_t)stream) != cudaSuccess)
         return EXL3_ERR_CUDA;
     return run_gemv(x, trellis, suh, svh, y, m, k, n, K, scratch, kNoAllocScratchBytes,
                     (cudaStream_t)stream);

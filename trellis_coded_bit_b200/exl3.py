@@ -145,6 +145,23 @@ def _ptr_or_none(t, dtype, name):
     return None if t is None else _dev(t, dtype, name)
 
 
+def _check_layer_shapes(x, trellis, suh, svh, K, y):
+    """Sizes of a layer's tensors against (m, k, n, K), checked before the C
+    call so that an undersized tensor never reaches a kernel."""
+    if x.dim() != 2:
+        raise ValueError("x must be m x k")
+    m, k = x.shape
+    n = svh.numel()
+    if suh.numel() != k:
+        raise ValueError("suh must have k = %d elements, has %d" % (k, suh.numel()))
+    if k % 16 or n % 16 or trellis.numel() != (k // 16) * (n // 16) * 16 * int(K):
+        raise ValueError("trellis must have (k/16)(n/16)16K = %d words for k=%d, n=%d, K=%d, has %d"
+                         % ((k // 16) * (n // 16) * 16 * int(K), k, n, int(K), trellis.numel()))
+    if y is not None and tuple(y.shape) != (m, n):
+        raise ValueError("y must be m x n = %d x %d, is %s" % (m, n, tuple(y.shape)))
+    return m, k, n
+
+
 # ----------------------------------------------------------------- calls ---
 
 def exl3_hadamard(x, y=None, pre=None, post=None, stream=None):
@@ -183,8 +200,7 @@ def new_workspace(nbytes, device=None):
 
 
 def _linear(fn, name, x, trellis, suh, svh, K, y, workspace, stream):
-    m, k = x.shape
-    n = svh.numel()
+    m, k, n = _check_layer_shapes(x, trellis, suh, svh, K, y)
     if y is None:
         y = torch.empty((m, n), dtype=torch.float16, device=x.device)
     if workspace is None:
@@ -208,7 +224,7 @@ def _linear_array(layers, m):
     for i, (x, trellis, suh, svh, K, y) in enumerate(layers):
         if x.shape[0] != m:
             raise ValueError("every layer of a multi call has the same batch size m")
-        k, n = x.shape[1], svh.numel()
+        _, k, n = _check_layer_shapes(x, trellis, suh, svh, K, y)
         if y is None:
             y = torch.empty((m, n), dtype=torch.float16, device=x.device)
         arr[i] = Exl3Linear(_dev(x, torch.float16, "x"), _dev(trellis, torch.uint16, "trellis"),
@@ -260,8 +276,7 @@ def exl3_gemv_noalloc_max_scratch():
 def exl3_gemv_noalloc(x, trellis, suh, svh, K, y, stream=None):
     """exl3_gemv without a workspace: the library's own fixed scratch array is
     used, for callers that cannot allocate device memory (y must be given)."""
-    m, k = x.shape
-    n = svh.numel()
+    m, k, n = _check_layer_shapes(x, trellis, suh, svh, K, y)
     _check(load().exl3_gemv_noalloc(_dev(x, torch.float16, "x"), _dev(trellis, torch.uint16, "trellis"),
                                     _dev(suh, torch.float16, "suh"), _dev(svh, torch.float16, "svh"),
                                     _dev(y, torch.float16, "y"), m, k, n, int(K), _stream(stream)),
