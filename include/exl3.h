@@ -186,8 +186,9 @@ exl3_status exl3_gemv_noalloc(const void *x, const uint16_t *trellis, const void
  * exl3_gemm -- the linear layer on the tensor cores (tcgen05 / TMEM), any
  * m >= 1, tuned for m >= 64 ([GEMM] section GEMM内核: Hadamard rotation of the
  * input, then the dequantising matmul; the kernel map picks tiles by shape).
- * n must be a multiple of 256 (EXL3_ERR_UNSUPPORTED otherwise).  The kernel
- * is persistent (one CTA per SM) and splits the work evenly over the CTAs by
+ * n is any multiple of 128: for n = 256j + 128 the last output tile carries
+ * 128 columns (its other half is computed from stale bytes and not stored).
+ * The kernel is persistent (one CTA per SM) and splits the work evenly over the CTAs by
  * (256 x 256 output tile, 64-channel k block) units, so a tile can be shared
  * by several CTAs; their fp32 partial sums meet in the workspace and are
  * added in a fixed order, so results are deterministic.  For m <= 64 the
@@ -207,6 +208,21 @@ size_t exl3_gemm_workspace_size(int64_t m, int64_t k, int64_t n, int K);
 exl3_status exl3_gemm(const void *x, const uint16_t *trellis, const void *suh, const void *svh,
                       void *y, int64_t m, int64_t k, int64_t n, int K, void *workspace,
                       size_t workspace_bytes, void *stream);
+
+/*
+ * exl3_matmul -- the layer for any m >= 1 with the kernel chosen inside the
+ * library ([GEMM] section GEMM内核: a kernel map picks the kernel from the
+ * problem shape; section 小批量GEMV: the decode-phase small batches are
+ * bandwidth bound and take the GEMV): m <= 16 runs exl3_gemv, larger m runs
+ * exl3_gemm.  Arguments, layout and errors as those two calls.
+ * `workspace` must hold exl3_matmul_workspace_size(m, k, n, K) bytes, the
+ * size of the path that m selects (zero-filled once after allocation, as
+ * for exl3_gemv / exl3_gemm).  Results are those of the selected call.
+ */
+size_t exl3_matmul_workspace_size(int64_t m, int64_t k, int64_t n, int K);
+exl3_status exl3_matmul(const void *x, const uint16_t *trellis, const void *suh, const void *svh,
+                        void *y, int64_t m, int64_t k, int64_t n, int K, void *workspace,
+                        size_t workspace_bytes, void *stream);
 
 /*
  * exl3_encode -- tail-biting trellis encoding of a weight matrix: for every

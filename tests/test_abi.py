@@ -66,7 +66,7 @@ def _gemv(fn, x=A, t=B, suh=C, svh=D, y=E, m=1, k=256, n=256, K=4, ws=None, wsb=
     return getattr(lib, fn)(x, t, suh, svh, y, m, k, n, K, ws, wsb, None)
 
 
-@pytest.mark.parametrize("fn", ["exl3_gemv", "exl3_gemm"])
+@pytest.mark.parametrize("fn", ["exl3_gemv", "exl3_gemm", "exl3_matmul"])
 def test_linear_argument_errors(fn):
     inv = exl3.EXL3_ERR_INVALID_ARG
     assert _gemv(fn, x=None) == inv
@@ -93,6 +93,25 @@ def test_workspace_sizes():
     assert lib.exl3_gemv_workspace_size(17, 4096, 4096, 4) == 0
     assert lib.exl3_gemv_workspace_size(1, 100, 4096, 4) == 0
     assert lib.exl3_gemm_workspace_size(2048, 8192, 28672, 3) >= 2048 * 8192 * 2
+
+
+def test_matmul_dispatch_and_gemm_tail_sizes():
+    # exl3_matmul picks the GEMV for m <= 16 and the GEMM above: its workspace
+    # size is that of the path m selects, and its workspace errors are that
+    # path's
+    lib = exl3.load()
+    for m in (1, 9, 16):
+        assert lib.exl3_matmul_workspace_size(m, 4096, 1024, 4) == lib.exl3_gemv_workspace_size(m, 4096, 1024, 4)
+    for m in (17, 32, 2048):
+        assert lib.exl3_matmul_workspace_size(m, 4096, 1024, 4) == lib.exl3_gemm_workspace_size(m, 4096, 1024, 4)
+    assert _gemv("exl3_matmul", m=16, ws=None) == exl3.EXL3_ERR_WORKSPACE
+    assert _gemv("exl3_matmul", m=32, ws=None) == exl3.EXL3_ERR_WORKSPACE
+    assert _gemv("exl3_matmul", m=32, ws=A, wsb=16) == exl3.EXL3_ERR_WORKSPACE
+    # the GEMM takes n = 256j + 128 (a half-width last tile)
+    for n in (128, 384, 1152):
+        assert lib.exl3_gemm_workspace_size(32, 1024, n, 3) > 0
+    assert lib.exl3_gemm_workspace_size(32, 1024, 200, 3) == 0
+    assert _gemv("exl3_gemm", m=32, n=384, ws=A, wsb=16) == exl3.EXL3_ERR_WORKSPACE  # not UNSUPPORTED
 
 
 def test_hadamard_and_decode_argument_errors():

@@ -100,10 +100,16 @@ def test_gemv_guards(m, k, n, K):
 
 
 @pytest.mark.parametrize("m,k,n,K", [(1, 128, 256, 3), (33, 512, 256, 5), (64, 256, 512, 1), (65, 128, 256, 2),
-                                     (200, 384, 768, 8)])
+                                     (200, 384, 768, 8), (32, 512, 384, 3), (130, 256, 128, 4)])
 def test_gemm_guards(m, k, n, K):
     layer = inputs.make_layer(m, k, n, K, seed=8200 + m + K)
     _linear_guarded(exl3.exl3_gemm, exl3.exl3_gemm_workspace_size, layer)
+
+
+@pytest.mark.parametrize("m", [3, 40])
+def test_matmul_guards(m):
+    layer = inputs.make_layer(m, 256, 384, 4, seed=8250 + m)
+    _linear_guarded(exl3.exl3_matmul, exl3.exl3_matmul_workspace_size, layer)
 
 
 def test_gemv_multi_guards():

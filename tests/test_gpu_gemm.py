@@ -115,3 +115,26 @@ def test_gemm_small_m_agrees_with_gemv_halves():
         yv = yv.cpu().numpy().astype(np.float64)
         ok, err, bound = within_tolerance(yg[rows], yv)
         assert ok, (h, err, bound)
+
+
+@pytest.mark.parametrize("m,k,n,K", [(32, 1024, 384, 3), (32, 2048, 1152, 4), (17, 512, 128, 2),
+                                     (200, 512, 384, 5), (64, 1024, 640, 8)])
+def test_gemm_half_width_last_tile(m, k, n, K):
+    # n = 256j + 128: the last output tile carries 128 columns; every column
+    # must match the oracle (guard regions around y: tests/test_gpu_canary.py)
+    layer = inputs.make_layer(m, k, n, K, seed=6500 + m + n + K)
+    y, _ = run_gemm(layer)
+    check(layer, y)
+
+
+@pytest.mark.parametrize("m", [1, 16, 17, 32, 65])
+def test_matmul_dispatch_matches_the_oracle(m):
+    # exl3_matmul runs the GEMV for m <= 16 and the GEMM above; both must give
+    # the layer to the stated tolerance, n = 384 included
+    k, n, K = 1024, 384, 3
+    layer = inputs.make_layer(m, k, n, K, seed=6600 + m)
+    ws = exl3.new_workspace(exl3.exl3_matmul_workspace_size(m, k, n, K))
+    y = exl3.exl3_matmul(dev(layer.x), dev(layer.trellis), dev(layer.suh), dev(layer.svh), K, workspace=ws)
+    torch.cuda.synchronize()
+    assert exl3.exl3_workspace_status(ws) == exl3.EXL3_OK
+    check(layer, y.cpu().numpy().astype(np.float64))

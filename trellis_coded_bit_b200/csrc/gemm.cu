@@ -481,9 +481,12 @@ __device__ __forceinline__ bool gemm_epilogue(const GemmParams &p, GemmBars &bar
         }
     }
     if (finish) {
+        // the last tile of n = 256j + 128 carries 128 columns: its other half
+        // holds results of stale weights and is not stored
+        const int halves = (tn + 1) * kBN > p.n ? 1 : kBN / 128;
         for (int mt = 0; mt < mt_count; ++mt) {
             const int row = tm * kBM * kMT + mt * kBM + erow;
-            for (int hb = 0; hb < kBN / 128; ++hb) {
+            for (int hb = 0; hb < halves; ++hb) {
                 const uint32_t col0 = (uint32_t)(mt * kBN + hb * 128);
                 // 32-point butterflies on each 32-column chunk, written back to TMEM
 #pragma unroll 1
@@ -638,8 +641,10 @@ __device__ __forceinline__ bool gemm_epilogue_wa(const GemmParams &p, GemmBars &
         }
     }
     if (finish) {
+        // the last tile of n = 256j + 128 carries only channel half 0
+        const int fchunks = (tn + 1) * kBN > p.n ? nchunks / 2 : nchunks;
 #pragma unroll 1
-        for (int cc = 0; cc < nchunks; ++cc) {
+        for (int cc = 0; cc < fchunks; ++cc) {
             const int h = (32 * cc) / nb, b0 = 32 * cc - h * nb;
             uint32_t r[32];
             EXL3_TMEM_LD32(tmem + lane_base + (uint32_t)(32 * cc), r);
@@ -786,11 +791,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmParams 
                     break;
                 }
                 unsigned char *dst = tring + s * kTrBytes;
-                mbar_arrive_expect_tx(&bars.tfull[s], (uint32_t)kTrBytes);
+                // the last tile of n = 256j + 128 has 8 trellis tiles per tile
+                // row, not 16; the decoders decode stale bytes for the rest
+                const int row_bytes = (tn + 1) * kBN > p.n ? kTileRowBytes / 2 : kTileRowBytes;
+                mbar_arrive_expect_tx(&bars.tfull[s], (uint32_t)((kBK / 16) * row_bytes));
                 const uint16_t *src = p.trellis + (int64_t)kb * (kBK / 16) * row_words + (int64_t)tn * 16 * 16 * K;
 #pragma unroll
                 for (int r = 0; r < kBK / 16; ++r)
-                    bulk_g2s(dst + r * kTileRowBytes, src + r * row_words, kTileRowBytes, &bars.tfull[s]);
+                    bulk_g2s(dst + r * kTileRowBytes, src + r * row_words, (uint32_t)row_bytes, &bars.tfull[s]);
                 issued = i + 1;
                 if (++kb == (int)KB) {
                     kb = 0;
@@ -932,6 +940,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmParams 
 
 // ------------------------------------------------------------- dispatch ---
 
+constexpr size_t kGemmSyncArea = 64 * 1024;
+
 struct GemmPlan {
     int64_t tiles, units;
     int tiles_n, kb_count, ctas;
@@ -942,7 +952,7 @@ static GemmPlan gemm_plan(int64_t m, int64_t k, int64_t n, int sms)
 {
     GemmPlan pl;
     const int64_t tiles_m = (m + kBM * kMT - 1) / (kBM * kMT);
-    pl.tiles_n = (int)(n / kBN);
+    pl.tiles_n = (int)((n + kBN - 1) / kBN);  // n = 256j + 128: a half-width last tile
     pl.tiles = tiles_m * pl.tiles_n;
     pl.kb_count = (int)(k / kBK);
     pl.units = pl.tiles * pl.kb_count;
@@ -953,6 +963,10 @@ static GemmPlan gemm_plan(int64_t m, int64_t k, int64_t n, int sms)
     pl.ctas = (int)(cap < sms ? cap : sms);
     pl.counters = 256;
     pl.xt = (pl.counters + (size_t)pl.tiles * 4 + 1023) / 1024 * 1024;
+    // data only from 64 KB on: the words below (status, counters) are zero
+    // after every call of either kind, so one workspace can serve GEMV and
+    // GEMM calls of any shapes in turn
+    pl.xt = pl.xt > kGemmSyncArea ? pl.xt : kGemmSyncArea;
     pl.partials = pl.xt + (size_t)(tiles_m * kBM * kMT) * (size_t)k * 2;
     pl.total = pl.partials + (size_t)2 * pl.ctas * kPartialFloats * 4;
     return pl;
@@ -974,7 +988,7 @@ static exl3_status launch_gemm_t(const GemmParams &p, cudaStream_t stream)
 
 extern "C" size_t exl3_gemm_workspace_size(int64_t m, int64_t k, int64_t n, int K)
 {
-    if (m < 1 || k < 128 || n < 256 || (k % 128) || (n % 256) || K < 1 || K > 8)
+    if (m < 1 || k < 128 || n < 128 || (k % 128) || (n % 128) || K < 1 || K > 8)
         return 0;
     return exl3::gemm_plan(m, k, n, exl3::num_sms()).total;
 }
@@ -987,8 +1001,6 @@ extern "C" exl3_status exl3_gemm(const void *x, const uint16_t *trellis, const v
     const exl3_status st = check_linear_args(x, trellis, suh, svh, y, m, k, n, K);
     if (st != EXL3_OK)
         return st;
-    if (n % kBN)
-        return EXL3_ERR_UNSUPPORTED;
     const GemmPlan pl = gemm_plan(m, k, n, num_sms());
     if (pl.units * (int64_t)pl.ctas >= ((int64_t)1 << 32))
         return EXL3_ERR_UNSUPPORTED;  // split the call along m (about 10^14 multiply-adds per call)

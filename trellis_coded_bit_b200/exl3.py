@@ -25,6 +25,7 @@ EXPORTED = ["exl3_status_string", "exl3_version", "exl3_hadamard", "exl3_decode_
             "exl3_gemv_workspace_size", "exl3_gemv", "exl3_gemv_multi_workspace_size", "exl3_gemv_multi",
             "exl3_gemv_noalloc_max_scratch",
             "exl3_gemv_noalloc", "exl3_gemm_workspace_size", "exl3_gemm",
+            "exl3_matmul_workspace_size", "exl3_matmul",
             "exl3_encode_workspace_size", "exl3_encode", "exl3_udu_workspace_size", "exl3_udu",
             "exl3_ldlq_workspace_size", "exl3_ldlq",
             "exl3_workspace_status", "exl3_set_launch_flags", "exl3_launch_flags",
@@ -73,10 +74,10 @@ def load(build_if_needed=True):
         lib.exl3_hadamard.restype = ci
         lib.exl3_decode_tiles.argtypes = [vp, vp, i64, i64, ci, vp]
         lib.exl3_decode_tiles.restype = ci
-        for name in ("exl3_gemv_workspace_size", "exl3_gemm_workspace_size"):
+        for name in ("exl3_gemv_workspace_size", "exl3_gemm_workspace_size", "exl3_matmul_workspace_size"):
             getattr(lib, name).argtypes = [i64, i64, i64, ci]
             getattr(lib, name).restype = sz
-        for name in ("exl3_gemv", "exl3_gemm"):
+        for name in ("exl3_gemv", "exl3_gemm", "exl3_matmul"):
             getattr(lib, name).argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, ci, vp, sz, vp]
             getattr(lib, name).restype = ci
         lib.exl3_gemv_multi_workspace_size.argtypes = [ctypes.POINTER(Exl3Linear), ci, i64]
@@ -193,6 +194,10 @@ def exl3_gemm_workspace_size(m, k, n, K):
     return int(load().exl3_gemm_workspace_size(m, k, n, K))
 
 
+def exl3_matmul_workspace_size(m, k, n, K):
+    return int(load().exl3_matmul_workspace_size(m, k, n, K))
+
+
 def new_workspace(nbytes, device=None):
     """Zero-filled workspace buffer (uint8) of at least nbytes, 256-byte aligned."""
     return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8,
@@ -287,6 +292,12 @@ def exl3_gemv_noalloc(x, trellis, suh, svh, K, y, stream=None):
 def exl3_gemm(x, trellis, suh, svh, K, y=None, workspace=None, stream=None):
     """The same layer on the tensor cores, any m (tuned for m >= 64)."""
     return _linear(load().exl3_gemm, "exl3_gemm", x, trellis, suh, svh, K, y, workspace, stream)
+
+
+def exl3_matmul(x, trellis, suh, svh, K, y=None, workspace=None, stream=None):
+    """The layer for any m, the kernel chosen by the library (GEMV for m <= 16,
+    tensor-core GEMM above)."""
+    return _linear(load().exl3_matmul, "exl3_matmul", x, trellis, suh, svh, K, y, workspace, stream)
 
 
 def exl3_encode_workspace_size(k, n, K):
