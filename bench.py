@@ -5,14 +5,18 @@ Default workload: the Llama-3.1-8B decode GEMV set -- m = 1, K in
 {2, 3, 4, 6, 8} x the four layer shapes (4096x4096, 4096x1024, 4096x14336,
 14336x4096), 20 layers, 398 MB of trellis in total (larger than the 126 MB
 L2, so every step streams the weights from HBM).  One step runs every layer
-once through exl3_gemv; the metric is algorithmic HBM GB/s (trellis + x + y +
-suh + svh bytes over time).  The prefill GEMM (m = 2048, 8192x28672, K = 3)
-is reported beside it in TFLOP/s.
+once through one exl3_gemv_multi call; the metric is algorithmic HBM GB/s
+(trellis + x + y + suh + svh bytes over time).  The prefill GEMM (m = 2048,
+8192x28672, K = 3) is reported beside it in TFLOP/s, with line items for the
+single PR1 layer, the 70B small-batch sweep, prefill at m = 512 and 8192, the
+70B layer stack and the offline encoder.
 
 Contract: `python bench.py --gpus N --steps K --warmup W` prints one JSON line
 on rank 0.  Under torchrun each rank runs its own replica of the workload
 (weak scaling, no collective in the data path); time = max over ranks.
-`--impl reference` times the fp64 CPU oracle on a bounded sample instead.
+`--impl reference` times the fp64 CPU oracle instead, on a fixed bounded
+sample of the same workload (every layer's first column blocks), and reports
+exactly what it timed.
 """
 import argparse
 import json
@@ -44,6 +48,7 @@ def parse():
     ap.add_argument("--no-gemm", action="store_true", help="skip the m=2048 GEMM line item")
     ap.add_argument("--no-stack", action="store_true", help="skip the 70B layer-stack line items")
     ap.add_argument("--no-encode", action="store_true", help="skip the trellis-encoder line item")
+    ap.add_argument("--no-items", action="store_true", help="skip the PR1 and small-batch sweep line items")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--profile", default=None,
@@ -255,27 +260,49 @@ def make_layers():
 
 # ------------------------------------------------------------- reference ---
 
+def reference_sample(L, threads):
+    """One step of the reference arm: the first `threads` 128-column blocks
+    (full k, all batches) of layer L through the fp64 oracle on all host
+    threads.  Returns (seconds, algorithmic bytes)."""
+    import oracle
+
+    b1 = min(L.n // 128, threads)
+    t0 = time.perf_counter()
+    oracle.linear(L.x, L.trellis, L.suh, L.svh, L.K, col_blocks=(0, b1), threads=threads)
+    sec = time.perf_counter() - t0
+    cols = b1 * 128
+    return sec, L.k * cols * L.K // 8 + 2 * L.m * L.k + 2 * L.m * cols + 2 * L.k + 2 * cols
+
+
 def run_reference(args, rank):
     if rank != 0:
         return
+    import oracle
+
     layers = make_layers()
-    total_bytes = sum(layer_bytes(L.m, L.k, L.n, L.K) for L in layers)
-    for _ in range(args.warmup):
-        cpu_oracle_sample(layers[:1], 0.01)
-    vals = []
-    per = max(1.0, args.cpu_seconds / max(1, args.steps))
-    for _ in range(args.steps):
-        vals.append(cpu_oracle_sample(layers, per))
-    value = statistics.median(v["value"] for v in vals)
-    cb = dict(vals[0])
-    cb["value"] = value
-    cb.pop("seconds", None)
+    threads = oracle.threads_available()
+    for i in range(args.warmup):
+        reference_sample(layers[i % len(layers)], threads)
+    total_s, total_b = 0.0, 0
+    for i in range(args.steps):
+        sec, done = reference_sample(layers[i % len(layers)], threads)
+        total_s += sec
+        total_b += done
+    ms = total_s / args.steps * 1e3
+    value = total_b / total_s / 1e9
+    sample = ("step i: layer i mod 20 of the workload, its first %d 128-column blocks (full k, m = 1); %d "
+              "algorithmic bytes over %d steps in %.1f s; fp64 oracle with %d OpenMP threads; ms_per_step = "
+              "that time / steps" % (threads, total_b, args.steps, total_s, threads))
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": total_bytes / (value * 1e9) * 1e3, "higher_is_better": True,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD_NAME, "parallelism": "host cores, oracle"},
-            "cpu_baseline": cb,
+            "config": {"workload": WORKLOAD_NAME, "m": 1, "layers": len(layers),
+                       "trellis_bytes_per_step": total_b // max(1, args.steps),
+                       "l2": "host caches (the oracle runs on the host cores)",
+                       "timing": "host wall clock around each step's sample",
+                       "api": "oracle.linear (fp64 CPU definition)", "launch": "none",
+                       "parallelism": "host cores, oracle", "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -457,8 +484,19 @@ def run_ours(args, rank, world, local_rank):
     if not args.no_encode:
         encode_info = bench_encode(exl3, torch, stream)
         encode_info.append(bench_ldlq(exl3, torch, stream))
+    extra_gemm = None
     if not args.no_gemm:
         gemm_info = bench_gemm(exl3, torch, peaks, stream)
+        extra_gemm = [bench_gemm(exl3, torch, peaks, stream, m=mm) for mm in (512, 8192)]
+    items = None
+    if not args.no_items:
+        items = {"pr1": bench_layer_calls(exl3, torch, peaks, stream, 1, 4096, 4096, 4, inputs.seed_for(0, 0)),
+                 "small_batch_sweep": [bench_layer_calls(exl3, torch, peaks, stream, mm, k, n, K,
+                                                         inputs.seed_for(2, i), True)
+                                       for i, (k, n, K, mm) in enumerate(
+                                           [(k, n, K, mm) for (k, n) in ((8192, 28672), (28672, 8192))
+                                            for K in (2, 4) for mm in (1, 16)])]}
+        items["pr1"]["workload"] = "PR1: one linear layer 4096x4096, K=4, m=1, one exl3_gemv call per layer copy"
     stack_info = None
     if not args.no_stack:
         stack_info = [bench_layer_stack(exl3, torch, peaks, stream, mm) for mm in (1, 32)]
@@ -466,9 +504,9 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0:
         ms = total_ms / args.steps
         value = job_throughput(step_bytes, world, ms)
-        # the step is 20 exl3_gemv calls (rotation + gemv_kernel each) in one
-        # graph; the per-call launches overlap (programmatic dependent launch),
-        # so the step's own duration is the kernels' duration
+        # the step is one exl3_gemv_multi call (a rotation launch and one
+        # persistent main launch) in one graph, so the step's own duration is
+        # the kernels' duration
         achieved = step_bytes / (ms * 1e-3) / 1e9
         traffic = measured_step_traffic()
         sms = torch.cuda.get_device_properties(local_rank).multi_processor_count
@@ -512,6 +550,10 @@ def run_ours(args, rank, world, local_rank):
                 "clocks": clocks}
         if gemm_info is not None:
             line["gemm"] = gemm_info
+        if extra_gemm is not None:
+            line["gemm_more"] = extra_gemm
+        if items is not None:
+            line.update(items)
         if encode_info is not None:
             line["encode"] = encode_info
         if stack_info is not None:
@@ -540,9 +582,7 @@ def bench_layer_stack(exl3, torch, peaks, stream, m):
     specs = [(nm, mm, k, n, K) for (nm, mm, k, n, K, _o) in workloads.LAYER_STACK if mm == m]
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
     use_gemv = m <= 16
-    size = exl3.exl3_gemv_workspace_size if use_gemv else exl3.exl3_gemm_workspace_size
-    call = exl3.exl3_gemv if use_gemv else exl3.exl3_gemm
-    ws = exl3.new_workspace(max(size(m, k, n, K) for (_nm, _m, k, n, K) in specs))
+    ws = exl3.new_workspace(max(exl3.exl3_matmul_workspace_size(m, k, n, K) for (_nm, _m, k, n, K) in specs))
     D = []
     for i, (nm, mm, k, n, K) in enumerate(specs):
         L = inputs.make_layer(m, k, n, K, inputs.seed_for(4, i))
@@ -567,8 +607,9 @@ def bench_layer_stack(exl3, torch, peaks, stream, m):
                 mc(w, stream=stream)
     else:
         def one_pass():
+            # the library picks the kernel (exl3_matmul: the GEMM for m > 16)
             for x, t, suh, svh, K, y in D:
-                call(x, t, suh, svh, K, y=y, workspace=ws, stream=stream)
+                exl3.exl3_matmul(x, t, suh, svh, K, y=y, workspace=ws, stream=stream)
 
     with torch.cuda.stream(stream):
         for _ in range(2):
@@ -592,15 +633,60 @@ def bench_layer_stack(exl3, torch, peaks, stream, m):
     del g
     return {"workload": "llama3.1-70b decoder-layer linear stack + lm_head, m=%d (%s)" %
                         (m, "exl3_gemv_multi per dependency group: q/k/v, o, gate/up, down, lm_head"
-                         if use_gemv else "exl3_gemm per layer"),
+                         if use_gemv else "exl3_matmul per layer, which runs the GEMM at this m"),
             "layers": [nm for (nm, _m, _k, _n, _K) in specs], "us_per_pass": us,
             "algorithmic_bytes_per_pass": total_bytes, "gb_s": total_bytes / (us * 1e-6) / 1e9,
             "frac_of_hbm_peak": total_bytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"]}
 
 
-def bench_gemm(exl3, torch, peaks, stream):
-    """m = 2048 prefill GEMM, 8192 x 28672, K = 3: TFLOP/s vs the fp16 peak."""
-    m, k, n, K = 2048, 8192, 28672, 3
+def bench_layer_calls(exl3, torch, peaks, stream, m, k, n, K, seed, outliers=False):
+    """One layer at batch m through exl3_matmul (the GEMV for m <= 16, the
+    GEMM above), timed as a CUDA graph of calls that cycle over copies of the
+    layer's trellis which together exceed 4x L2, so that every call streams its
+    weights from HBM.  Returns microseconds per call, algorithmic GB/s and the
+    fraction of the measured HBM peak."""
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    L = inputs.make_layer(m, k, n, K, seed, outliers)
+    t0 = dev(L.trellis)
+    l2 = getattr(torch.cuda.get_device_properties(torch.cuda.current_device()), "L2_cache_size", 126 << 20)
+    copies = max(2, -(-4 * l2 // L.trellis.nbytes))
+    ts = [t0] + [t0.clone() for _ in range(copies - 1)]
+    x, suh, svh = dev(L.x), dev(L.suh), dev(L.svh)
+    y = torch.empty((m, n), dtype=torch.float16, device="cuda")
+    ws = exl3.new_workspace(exl3.exl3_matmul_workspace_size(m, k, n, K))
+
+    def calls():
+        for t in ts:
+            exl3.exl3_matmul(x, t, suh, svh, K, y=y, workspace=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        calls()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        calls()
+    reps = 5
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            g.replay()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / (reps * copies)
+    del g, ts
+    b = layer_bytes(m, k, n, K)
+    return {"m": m, "k": k, "n": n, "K": K, "us": us, "gb_s": b / (us * 1e-6) / 1e9,
+            "frac_of_hbm_peak": b / (us * 1e-6) / 1e9 / peaks["hbm_gbs"],
+            "path": "exl3_gemv" if m <= 16 else "exl3_gemm", "trellis_copies": copies}
+
+
+def bench_gemm(exl3, torch, peaks, stream, m=2048):
+    """Prefill GEMM at batch m, 8192 x 28672, K = 3: TFLOP/s vs the fp16 peak."""
+    k, n, K = 8192, 28672, 3
     L = inputs.make_layer(m, k, n, K, inputs.seed_for(3, 2))
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
     x, t, suh, svh = dev(L.x), dev(L.trellis), dev(L.suh), dev(L.svh)
@@ -628,7 +714,7 @@ def bench_gemm(exl3, torch, peaks, stream):
     tf = flops / (ms * 1e-3) / 1e12
     # fp16 dense peak equals the bf16 one on B200 (same tensor-core rate)
     peak = peaks["bf16_tflops"]
-    return {"workload": "llama3.1-70b gate/up prefill m=2048, 8192x28672, K=3", "ms": ms,
+    return {"workload": "llama3.1-70b gate/up prefill m=%d, 8192x28672, K=3" % m, "ms": ms,
             "tflops": tf, "peak_tflops": peak, "frac": tf / peak,
             "peak_source": peaks["source"] + " bf16 cuBLAS burst (fp16 rate is the same)"}
 
