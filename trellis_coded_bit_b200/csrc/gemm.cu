@@ -222,6 +222,20 @@ __device__ __forceinline__ void fence_proxy_async_smem()
                  : "r"(taddr), "r"((taddr) + 32u), "r"((taddr) + 64u), "r"((taddr) + 96u)                  \
                  : "memory")
 
+// Four 8-column stores of v[0..31] at taddr, taddr + 32, + 64, + 96 (no wait).
+#define EXL3_TMEM_ST8X4(taddr, v)                                                                         \
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%4,%5,%6,%7,%8,%9,%10,%11};\n"              \
+                 "tcgen05.st.sync.aligned.32x32b.x8.b32 [%1], {%12,%13,%14,%15,%16,%17,%18,%19};\n"        \
+                 "tcgen05.st.sync.aligned.32x32b.x8.b32 [%2], {%20,%21,%22,%23,%24,%25,%26,%27};\n"        \
+                 "tcgen05.st.sync.aligned.32x32b.x8.b32 [%3], {%28,%29,%30,%31,%32,%33,%34,%35};\n"        \
+                 ::"r"(taddr), "r"((taddr) + 32u), "r"((taddr) + 64u), "r"((taddr) + 96u),                \
+                 "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),   \
+                 "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),          \
+                 "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),        \
+                 "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),        \
+                 "r"(v[29]), "r"(v[30]), "r"(v[31])                                                        \
+                 : "memory")
+
 __device__ __forceinline__ void tmem_wait_st()
 {
     asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
@@ -481,14 +495,40 @@ __device__ __forceinline__ bool gemm_epilogue(const GemmParams &p, GemmBars &bar
         }
     }
     if (finish) {
-        // the last tile of n = 256j + 128 carries 128 columns: its other half
-        // holds results of stale weights and is not stored
+        // H128 = H4 (x) H32 on each 128-column half: first the 4-point stage
+        // across the four 32-column chunks (eight columns of each per TMEM
+        // round trip), then per chunk the 32-point butterflies in registers,
+        // svh/sqrt(128) and fp16.  A chunk is 64 contiguous bytes of the row
+        // the lane holds; a 4 x 4 exchange of 16-byte pieces within each group
+        // of four lanes then lets the group store 64 contiguous bytes of one
+        // row per instruction (8 rows per warp store instead of 32).
+        // The last tile of n = 256j + 128 carries 128 columns: its other half
+        // holds results of stale weights and is not stored.
         const int halves = (tn + 1) * kBN > p.n ? 1 : kBN / 128;
+        const int gi = lane & 3;                 // piece this lane stores
+        const int grow = erow - gi;              // first row of the lane's group
         for (int mt = 0; mt < mt_count; ++mt) {
-            const int row = tm * kBM * kMT + mt * kBM + erow;
+            const int row0 = tm * kBM * kMT + mt * kBM + grow;
             for (int hb = 0; hb < halves; ++hb) {
                 const uint32_t col0 = (uint32_t)(mt * kBN + hb * 128);
-                // 32-point butterflies on each 32-column chunk, written back to TMEM
+#pragma unroll 1
+                for (int o = 0; o < 4; ++o) {
+                    uint32_t w[32];  // [chunk c][8 columns]
+                    const uint32_t ta = tmem + lane_base + col0 + 8 * o;
+                    EXL3_TMEM_LD8X4(ta, w);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float a0 = __uint_as_float(w[e]), a1 = __uint_as_float(w[8 + e]);
+                        const float a2 = __uint_as_float(w[16 + e]), a3 = __uint_as_float(w[24 + e]);
+                        const float s01 = a0 + a1, d01 = a0 - a1, s23 = a2 + a3, d23 = a2 - a3;
+                        w[e] = __float_as_uint(s01 + s23);
+                        w[8 + e] = __float_as_uint(d01 + d23);
+                        w[16 + e] = __float_as_uint(s01 - s23);
+                        w[24 + e] = __float_as_uint(d01 - d23);
+                    }
+                    EXL3_TMEM_ST8X4(ta, w);
+                }
+                tmem_wait_st();
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     uint32_t r[32];
@@ -498,47 +538,47 @@ __device__ __forceinline__ bool gemm_epilogue(const GemmParams &p, GemmBars &bar
                     for (int i = 0; i < 32; ++i)
                         v[i] = __uint_as_float(r[i]);
                     fwht32(v);
+                    const int ncol0 = tn * kBN + hb * 128 + 32 * c;
+                    // piece q (columns 8q .. 8q + 7 of the chunk) as 4 words
+                    uint32_t pc[4][4];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        r[i] = __float_as_uint(v[i]);
-                    EXL3_TMEM_ST32(tmem + lane_base + col0 + 32 * c, r);
-                    tmem_wait_st();
-                }
-                // 4-point stage across the chunks, scale, fp16, store
-#pragma unroll 1
-                for (int o = 0; o < 4; ++o) {
-                    uint32_t w[32];  // [chunk c][8 columns]
-                    EXL3_TMEM_LD8X4(tmem + lane_base + col0 + 8 * o, w);
-                    if (row < p.m) {
+                    for (int q = 0; q < 4; ++q) {
+                        const uint4 sv4 = *reinterpret_cast<const uint4 *>(p.svh + ncol0 + 8 * q);
+                        const __half2 *sv = reinterpret_cast<const __half2 *>(&sv4);
+                        const float sc = 0.08838834764831845f;
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            const int ncol = tn * kBN + hb * 128 + 32 * c + 8 * o;
-                            const uint4 sv4 = *reinterpret_cast<const uint4 *>(p.svh + ncol);
-                            const __half2 *sv = reinterpret_cast<const __half2 *>(&sv4);
-                            uint32_t pk[4];
-#pragma unroll
-                            for (int e = 0; e < 8; e += 2) {
-                                float z[2];
-#pragma unroll
-                                for (int d = 0; d < 2; ++d) {
-                                    const float a0 = __uint_as_float(w[0 + e + d]);
-                                    const float a1 = __uint_as_float(w[8 + e + d]);
-                                    const float a2 = __uint_as_float(w[16 + e + d]);
-                                    const float a3 = __uint_as_float(w[24 + e + d]);
-                                    const float s01 = a0 + a1, d01 = a0 - a1, s23 = a2 + a3,
-                                                d23 = a2 - a3;
-                                    // H4 row c: c=0 (+,+,+,+) c=1 (+,-,+,-) c=2 (+,+,-,-) c=3 (+,-,-,+)
-                                    z[d] = c == 0 ? s01 + s23 : c == 1 ? d01 + d23 : c == 2 ? s01 - s23 : d01 - d23;
-                                }
-                                const float sc = 0.08838834764831845f;
-                                __half2 h = __floats2half2_rn(z[0] * sc * __low2float(sv[e >> 1]),
-                                                              z[1] * sc * __high2float(sv[e >> 1]));
-                                pk[e >> 1] = *reinterpret_cast<uint32_t *>(&h);
-                            }
-                            *reinterpret_cast<uint4 *>(p.y + (int64_t)row * p.n + ncol) =
-                                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        for (int e = 0; e < 4; ++e) {
+                            __half2 h = __floats2half2_rn(v[8 * q + 2 * e] * sc * __low2float(sv[e]),
+                                                          v[8 * q + 2 * e + 1] * sc * __high2float(sv[e]));
+                            pc[q][e] = *reinterpret_cast<uint32_t *>(&h);
                         }
                     }
+                    // 4 x 4 exchange: afterwards slot s of lane 4g + i holds
+                    // piece i of row 4g + s
+#pragma unroll
+                    for (int b = 2; b >= 1; b >>= 1) {
+                        const bool hi = (lane & b) != 0;
+#pragma unroll
+                        for (int q0 = 0; q0 < 4; ++q0) {
+                            if (q0 & b)
+                                continue;
+                            const int q1 = q0 ^ b;
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const uint32_t send = hi ? pc[q0][e] : pc[q1][e];
+                                const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, b);
+                                if (hi)
+                                    pc[q0][e] = recv;
+                                else
+                                    pc[q1][e] = recv;
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int sr = 0; sr < 4; ++sr)
+                        if (row0 + sr < p.m)
+                            *reinterpret_cast<uint4 *>(p.y + (int64_t)(row0 + sr) * p.n + ncol0 + 8 * gi) =
+                                make_uint4(pc[sr][0], pc[sr][1], pc[sr][2], pc[sr][3]);
                 }
             }
         }
