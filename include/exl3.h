@@ -123,8 +123,10 @@ exl3_status exl3_gemv(const void *x, const uint16_t *trellis, const void *suh, c
  *   layers    HOST array of `count` descriptors (copied during the call; the
  *             pointers in it are device memory, laid out as for exl3_gemv).
  *   count     1 .. any; every 32 layers (in call order, any mix of K) run
- *             as one rotation launch plus one persistent launch, so the fixed
- *             cost of a launch is paid once, not per layer or per K.  The
+ *             as one persistent launch (preceded by one input-rotation
+ *             launch unless every CTA's share is short enough to rotate its
+ *             own inputs), so the fixed cost is paid once, not per layer or
+ *             per K.  The
  *             persistent launch splits its CTAs into one group per K (in
  *             proportion to the group's estimated cost), and a group's CTAs
  *             share out its work units evenly.
@@ -317,7 +319,10 @@ unsigned exl3_launch_flags(void);
 /*
  * exl3_workspace_status -- read (synchronously, on `stream`) the status word a
  * gemv/gemm call leaves in its workspace: EXL3_OK, or EXL3_ERR_TIMEOUT if a
- * bounded device wait ran out.  `clear` != 0 resets it to EXL3_OK.
+ * bounded device wait ran out.  `clear` != 0 resets it to EXL3_OK and zeroes
+ * the rest of the workspace's first 64 KiB (the arrival counters, which a
+ * call that timed out may leave nonzero), so the workspace can serve further
+ * calls.
  */
 exl3_status exl3_workspace_status(void *workspace, size_t workspace_bytes, int clear, void *stream);
 

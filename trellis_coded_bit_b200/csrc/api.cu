@@ -79,7 +79,10 @@ extern "C" exl3_status exl3_workspace_status(void *workspace, size_t workspace_b
     cudaStream_t s = (cudaStream_t)stream;
     if (cudaMemcpyAsync(&word, workspace, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess)
         return EXL3_ERR_CUDA;
-    if (clear && cudaMemsetAsync(workspace, 0, 4, s) != cudaSuccess)
+    // the sync area every gemv/gemm workspace starts with (status word,
+    // arrival counters)
+    const size_t sync = workspace_bytes < 65536 ? workspace_bytes : 65536;
+    if (clear && cudaMemsetAsync(workspace, 0, sync, s) != cudaSuccess)
         return EXL3_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess)
         return EXL3_ERR_CUDA;

@@ -4,11 +4,20 @@
 // bandwidth, so a dedicated GEMV path streams the quantised weights once).
 //
 // B200 design (the pages' consumer-GPU GEMV is prior art, not copied):
-//   * Two launches.  A rotation kernel computes x' = H(x .* suh)/sqrt(128)
-//     (fp32 butterflies, fp16 result) and writes it into the workspace as
-//     tensor-core B-fragment activation blocks (see below); the main kernel
-//     streams the weights and copies those blocks with them.
-//   * The main kernel is persistent and "stream-K" balanced.  One launch
+//   * The input rotation x' = H(x .* suh)/sqrt(128) (fp32 butterflies, fp16
+//     result) goes into the workspace as tensor-core B-fragment activation
+//     blocks (see below), which the main loop copies into shared memory with
+//     the weights.  When each CTA's unit range is short (single layers at
+//     small m, where the fixed cost of a call dominates) the call is ONE
+//     launch: after requesting its first weights every CTA rotates just the
+//     128-channel blocks its own range reads, and a CTA barrier is all the
+//     synchronisation.  Otherwise (long ranges: many layers, or m large
+//     enough that a CTA would rotate many blocks) a rotation kernel runs
+//     just before the main kernel, which is resident and streaming weights
+//     meanwhile (programmatic dependent launch).  Sharing that rotation over
+//     the main kernel's own warps behind a grid barrier measured slower on
+//     the 20-layer decode step (170.4 against 169.2 us per step back to back).
+//   * The kernel is persistent and "stream-K" balanced.  One launch
 //     serves every layer of an exl3_gemv_multi call (up to 32, any mix of K):
 //     its CTAs are split into one group per K, in proportion to the group's
 //     cost, so that each CTA runs the decode compiled for one K.  Within a
@@ -44,8 +53,9 @@
 //   * Each warp streams its units through its own 3-deep cp.async ring in
 //     shared memory (8 tiles padded against bank conflicts, plus the unit's
 //     activation block), loaded by 16-byte copies spread over the lanes.
-//   * With EXL3_LAUNCH_PDL the main kernel requests its first weights before
-//     it waits for the rotation kernel (griddepcontrol).
+//   * With EXL3_LAUNCH_PDL the kernel is resident and requests its first
+//     weights while the preceding kernel drains, and waits for it
+//     (griddepcontrol) only before it reads x.
 #include <cuda_fp16.h>
 
 #include "exl3_device.cuh"
@@ -78,67 +88,6 @@ __host__ __device__ inline int gemv_mg(int64_t m)
     return m > 8 ? 2 : 1;
 }
 
-// ------------------------------------------------------ rotation kernel ---
-
-struct GemvRotLayer {
-    const __half *x;
-    const __half *suh;
-    unsigned char *acts;
-    int k;
-    int64_t job_begin;  // first job of this layer
-};
-
-constexpr int kGemvRotMaxLayers = 32;  // at least the main launch's layer limit
-
-struct GemvRotParams {
-    GemvRotLayer L[kGemvRotMaxLayers];
-    int count, m;
-    int64_t jobs;
-};
-
-// One warp per (layer, batch, 128-channel block): lane l rotates channels
-// 4l .. 4l+3 and writes them as one 16-byte piece of the activation blocks.
-__global__ void __launch_bounds__(256) gemv_rotate_kernel(const GemvRotParams rp)
-{
-    grid_dep_wait();    // x may come from the preceding kernel
-    grid_dep_launch();  // the main kernel may start streaming weights meanwhile
-    const int lane = threadIdx.x & 31;
-    const int m = rp.m;
-    const int MG = gemv_mg(m);
-    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    const float s128 = 0.08838834764831845f;
-    int l = 0;
-    for (int64_t job = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); job < rp.jobs; job += warps) {
-        while (l + 1 < rp.count && job >= rp.L[l + 1].job_begin)
-            ++l;
-        const GemvRotLayer &L = rp.L[l];
-        const int k = L.k, nblk = k / 128;
-        const int64_t lj = job - L.job_begin;
-        const int b = (int)(lj / nblk), blk = (int)(lj - (int64_t)b * nblk);
-        const int c = blk * 128 + lane * 4;
-        const uint2 sr = *reinterpret_cast<const uint2 *>(L.suh + c);
-        const uint2 r0 = *reinterpret_cast<const uint2 *>(L.x + (int64_t)b * k + c);
-        const __half2 *sv = reinterpret_cast<const __half2 *>(&sr);
-        const __half2 *x0 = reinterpret_cast<const __half2 *>(&r0);
-        float v[4] = {__low2float(x0[0]) * __low2float(sv[0]), __high2float(x0[0]) * __high2float(sv[0]),
-                      __low2float(x0[1]) * __low2float(sv[1]), __high2float(x0[1]) * __high2float(sv[1])};
-        warp_fwht128(v);
-        uint32_t d[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const uint32_t h = (uint32_t)__half_as_ushort(__float2half_rn(v[e] * s128));
-            d[e] = h | (h << 16);
-        }
-        // channels c .. c+3: tile row c / 16, rows r .. r+3 with r = c % 16
-        // (r = 8ks + 2t0, t0 even): entries (ks, g, t0) and (ks, g, t0 + 1)
-        const int tr = c >> 4, r = c & 15;
-        const int mg = b >> 3, g = b & 7;
-        unsigned char *dst = L.acts + ((int64_t)tr * MG + mg) * kGemvActBlock + (r >> 3) * 256 + g * 32 +
-                             ((r & 7) >> 1) * 8;
-        *reinterpret_cast<uint4 *>(dst) = make_uint4(d[0], d[1], d[2], d[3]);
-    }
-}
-
 // ---------------------------------------------------------- main kernel ---
 
 // One launch covers up to kGemvMaxLayers layers with the same m and any mix
@@ -151,9 +100,9 @@ constexpr int kGemvMaxLayers = 32;
 
 struct GemvLayer {
     const unsigned char *trellis;  // uint16 [k/16][n/16][16K]
-    const __half *svh;
+    const __half *x, *suh, *svh;
     __half *y;
-    const unsigned char *acts;  // activation blocks [k/16][MG][512 B]
+    unsigned char *acts;        // activation blocks [k/16][MG][512 B]
     float *partials;            // [n/128][max_seg][m][128]
     uint32_t *counters;         // [n/128]
     int64_t unit_begin;         // the layer's first unit within its group
@@ -182,6 +131,10 @@ struct GemvParams {
     GemvLayer L[kGemvMaxLayers];
     GemvGroup grp[8];
     int ngroups, m;
+    // Input rotation: rot_local != 0 -- every CTA rotates the 128-channel
+    // blocks its own unit range reads; 0 -- the rotation kernel launched just
+    // before has written every activation block.
+    int rot_local;
     Codebook cb;
     GemvMults mu;
 };
@@ -431,6 +384,65 @@ __device__ __forceinline__ void finish_block(const GemvLayer &L, int m, const fl
     }
 }
 
+// ------------------------------------------------------ input rotation ---
+
+// x' = H(x .* suh)/sqrt(128) for one 128-channel block `blk` of batch row b
+// of a layer with k input channels, by one warp: lane l rotates channels
+// 4l .. 4l+3 (fp32 butterflies, fp16 result) and writes them as one 16-byte
+// piece of the activation blocks `acts` (each value duplicated into both
+// halves of a word).
+__device__ __forceinline__ void rotate_block(const __half *x, const __half *suh, unsigned char *acts, int k,
+                                             int m, int b, int blk, int lane)
+{
+    const int MG = gemv_mg(m);
+    const int c = blk * 128 + lane * 4;
+    const uint2 sr = *reinterpret_cast<const uint2 *>(suh + c);
+    const uint2 r0 = *reinterpret_cast<const uint2 *>(x + (int64_t)b * k + c);
+    const __half2 *sv = reinterpret_cast<const __half2 *>(&sr);
+    const __half2 *x0 = reinterpret_cast<const __half2 *>(&r0);
+    float v[4] = {__low2float(x0[0]) * __low2float(sv[0]), __high2float(x0[0]) * __high2float(sv[0]),
+                  __low2float(x0[1]) * __low2float(sv[1]), __high2float(x0[1]) * __high2float(sv[1])};
+    warp_fwht128(v);
+    const float s128 = 0.08838834764831845f;
+    uint32_t d[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const uint32_t h = (uint32_t)__half_as_ushort(__float2half_rn(v[e] * s128));
+        d[e] = h | (h << 16);
+    }
+    // channels c .. c+3: tile row c / 16, rows r .. r+3 with r = c % 16
+    // (r = 8ks + 2t0, t0 even): entries (ks, g, t0) and (ks, g, t0 + 1)
+    const int tr = c >> 4, r = c & 15;
+    const int mg = b >> 3, g = b & 7;
+    unsigned char *dst =
+        acts + ((int64_t)tr * MG + mg) * kGemvActBlock + (r >> 3) * 256 + g * 32 + ((r & 7) >> 1) * 8;
+    *reinterpret_cast<uint4 *>(dst) = make_uint4(d[0], d[1], d[2], d[3]);
+}
+
+// Local rotation: the CTA rotates the blocks that hold the tile rows of its
+// own unit range [u0, u1), which the host guarantees to span at most two
+// column blocks: rows [r0, r1] of one, or rows [r0, TR) of the first and
+// [0, r1] of the second (possibly of the next layer).  CTAs whose ranges
+// share a block write the same bytes.  A CTA barrier afterwards makes the
+// blocks visible to the CTA's own copies.
+__device__ __forceinline__ void rotate_local(const GemvParams &p, int lb, int le, int64_t u0, int64_t u1,
+                                             int warp, int lane)
+{
+    int l0 = lb, c0 = 0, r0 = 0, l1 = lb, c1 = 0, r1 = 0;
+    gemv_locate(p, le, u0, l0, c0, r0);
+    gemv_locate(p, le, u1 - 1, l1, c1, r1);
+    const int m = p.m;
+    const bool one = l0 == l1 && c0 == c1;
+    // segment A: layer l0, blocks [a0, a1]; segment B: layer l1, blocks [0, b1]
+    const int a0 = r0 >> 3, a1 = one ? (r1 >> 3) : ((p.L[l0].tr_count - 1) >> 3);
+    const int nA = (a1 - a0 + 1) * m, nB = one ? 0 : ((r1 >> 3) + 1) * m;
+    for (int j = warp; j < nA + nB; j += kGemvWarps) {
+        const GemvLayer &L = p.L[j < nA ? l0 : l1];
+        const int jj = j < nA ? j : j - nA;
+        rotate_block(L.x, L.suh, L.acts, 16 * L.tr_count, m, jj % m, (j < nA ? a0 : 0) + jj / m, lane);
+    }
+}
+
 // The work of one CTA of a K group.  CTA c of the group's G owns the
 // contiguous unit range [cU/G, (c+1)U/G); its 8 warps take units u0 + w,
 // u0 + w + 8, ..., so that a CTA's concurrent loads stay within a few
@@ -538,9 +550,10 @@ __device__ __forceinline__ void gemv_cta(const GemvParams &p, const GemvGroup &g
     };
 
     // Prologue: the first kGemvDepth units' weights are requested before the
-    // wait for the rotation kernel (which writes the activation blocks; a
-    // no-op without PDL), their activations after it.  The ring's entries of
-    // absent batches are zeroed once; copies never touch them.
+    // wait for the preceding kernel (which may write x; a no-op without PDL),
+    // then the input rotation writes the activation blocks, and the units'
+    // activations are copied after it.  The ring's entries of absent batches
+    // are zeroed once; copies never touch them.
     const unsigned char *asrc0[kGemvDepth];
 #pragma unroll
     for (int d = 0; d < kGemvDepth; ++d) {
@@ -555,6 +568,10 @@ __device__ __forceinline__ void gemv_cta(const GemvParams &p, const GemvGroup &g
     __syncwarp();
     grid_dep_wait();
     grid_dep_launch();  // a dependent launch still waits for this grid to complete
+    if (p.rot_local) {
+        rotate_local(p, lb, le, u0, u1, warp, lane);
+        __syncthreads();
+    }
 #pragma unroll
     for (int d = 0; d < kGemvDepth; ++d)
         if (asrc0[d])
@@ -725,6 +742,7 @@ struct GemvPlan {
     int cb_begin[kGemvMaxLayers], max_seg[kGemvMaxLayers];  // by plan index
     size_t counters[kGemvMaxLayers], acts[kGemvMaxLayers], partials[kGemvMaxLayers];  // by call index
     size_t sync_bytes, total;
+    int rot_local;  // input rotation per CTA (1) or shared with a grid barrier (0)
 };
 
 // Relative time of one unit at m = 1 by K: each K group of the Llama-3.1-8B
@@ -838,6 +856,22 @@ static GemvPlan gemv_plan(const int64_t *k, const int64_t *n, const int *K, int 
     }
     pl.ctas = cta;
 
+    // Input rotation.  Per CTA, inside the one launch, when every CTA's range
+    // spans at most two column blocks (its length is at most the smallest
+    // tile-row count of its group) and touches few enough 128-channel blocks
+    // that each warp rotates at most two (range / 8 + 2 blocks, m rows each);
+    // otherwise by the rotation kernel, launched just before.
+    pl.rot_local = 1;
+    for (int q = 0; q < pl.ngroups; ++q) {
+        const GemvGroup &gr = pl.grp[q];
+        const int64_t range = (gr.units + gr.ctas - 1) / gr.ctas;
+        int64_t tr_min = INT64_MAX;
+        for (int i = gr.l_begin; i < gr.l_end; ++i)
+            tr_min = k[pl.order[i]] / 16 < tr_min ? k[pl.order[i]] / 16 : tr_min;
+        if (range > tr_min || (range / 8 + 2) * m > 2 * kGemvWarps)
+            pl.rot_local = 0;
+    }
+
     size_t off = 256;
     for (int l = 0; l < count; ++l) {
         pl.counters[l] = off;
@@ -891,8 +925,39 @@ size_t gemv_workspace_bytes(int64_t m, int64_t k, int64_t n, int sms)
     return most;
 }
 
-// Launches the rotation kernel over `count` (<= kGemvMaxLayers) layers:
-// layer l's activation blocks go to acts[l].
+// The rotation kernel, for launches whose CTA ranges are long: one warp per
+// (layer, batch row, 128-channel block) job, layer by layer.
+struct GemvRotLayer {
+    const __half *x, *suh;
+    unsigned char *acts;
+    int k;
+    int64_t job_begin;  // first job of this layer
+};
+
+struct GemvRotParams {
+    GemvRotLayer L[kGemvMaxLayers];
+    int count, m;
+    int64_t jobs;
+};
+
+__global__ void __launch_bounds__(256) gemv_rotate_kernel(const GemvRotParams rp)
+{
+    grid_dep_wait();    // x may come from the preceding kernel
+    grid_dep_launch();  // the main kernel may start streaming weights meanwhile
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    int l = 0;
+    for (int64_t job = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); job < rp.jobs; job += warps) {
+        while (l + 1 < rp.count && job >= rp.L[l + 1].job_begin)
+            ++l;
+        const GemvRotLayer &L = rp.L[l];
+        const int nblk = L.k / 128;
+        const int64_t lj = job - L.job_begin;
+        const int b = (int)(lj / nblk);
+        rotate_block(L.x, L.suh, L.acts, L.k, rp.m, b, (int)(lj - (int64_t)b * nblk), lane);
+    }
+}
+
 static exl3_status launch_rotation(const exl3_linear *const *layers, unsigned char *const *acts, int count,
                                    int64_t m, cudaStream_t stream)
 {
@@ -920,8 +985,8 @@ static exl3_status launch_rotation(const exl3_linear *const *layers, unsigned ch
     return launch_status();
 }
 
-// One rotation launch and one main launch over up to kGemvMaxLayers layers,
-// with the workspace region `ws` laid out by gemv_plan.
+// One launch over up to kGemvMaxLayers layers (two when the rotation runs as
+// its own kernel), with the workspace region `ws` laid out by gemv_plan.
 static exl3_status run_gemv_launch(const exl3_linear *const *layers, int count, int64_t m, unsigned char *ws,
                                    size_t ws_bytes, cudaStream_t stream)
 {
@@ -936,16 +1001,18 @@ static exl3_status run_gemv_launch(const exl3_linear *const *layers, int count, 
     const GemvPlan pl = gemv_plan(k, n, K, count, m, sms);
     if (!ws || !aligned16(ws) || ws_bytes < pl.total)
         return EXL3_ERR_WORKSPACE;
-
-    unsigned char *acts[kGemvMaxLayers];
-    for (int l = 0; l < count; ++l)
-        acts[l] = ws + pl.acts[l];
-    const exl3_status rs = launch_rotation(layers, acts, count, m, stream);
-    if (rs != EXL3_OK)
-        return rs;
+    if (!pl.rot_local) {
+        unsigned char *acts[kGemvMaxLayers];
+        for (int l = 0; l < count; ++l)
+            acts[l] = ws + pl.acts[l];
+        const exl3_status rs = launch_rotation(layers, acts, count, m, stream);
+        if (rs != EXL3_OK)
+            return rs;
+    }
 
     GemvParams p;
     p.m = (int)m;
+    p.rot_local = pl.rot_local;
     p.ngroups = pl.ngroups;
     for (int q = 0; q < pl.ngroups; ++q)
         p.grp[q] = pl.grp[q];
@@ -956,6 +1023,8 @@ static exl3_status run_gemv_launch(const exl3_linear *const *layers, int count, 
         const int l = pl.order[i];
         GemvLayer &L = p.L[i];
         L.trellis = reinterpret_cast<const unsigned char *>(layers[l]->trellis);
+        L.x = (const __half *)layers[l]->x;
+        L.suh = (const __half *)layers[l]->suh;
         L.svh = (const __half *)layers[l]->svh;
         L.y = (__half *)layers[l]->y;
         L.acts = ws + pl.acts[l];
