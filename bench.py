@@ -665,18 +665,22 @@ def bench_layer_calls(exl3, torch, peaks, stream, m, k, n, K, seed, outliers=Fal
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
         calls()
-    reps = 5
+    reps, rounds = 5, 5
     with torch.cuda.stream(stream):
         for _ in range(2):
             g.replay()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(reps):
-            g.replay()
-        e1.record(stream)
-    torch.cuda.synchronize()
-    us = e0.elapsed_time(e1) * 1e3 / (reps * copies)
+    per_round = []
+    for _ in range(rounds):  # the median round: one slow round (another job's burst) does not set it
+        with torch.cuda.stream(stream):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        per_round.append(e0.elapsed_time(e1) * 1e3 / (reps * copies))
+    us = sorted(per_round)[rounds // 2]
     del g, ts
     b = layer_bytes(m, k, n, K)
     return {"m": m, "k": k, "n": n, "K": K, "us": us, "gb_s": b / (us * 1e-6) / 1e9,
