@@ -581,7 +581,6 @@ def bench_layer_stack(exl3, torch, peaks, stream, m):
     646 MB of trellis, larger than L2)."""
     specs = [(nm, mm, k, n, K) for (nm, mm, k, n, K, _o) in workloads.LAYER_STACK if mm == m]
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
-    use_gemv = m <= 16
     ws = exl3.new_workspace(max(exl3.exl3_matmul_workspace_size(m, k, n, K) for (_nm, _m, k, n, K) in specs))
     D = []
     for i, (nm, mm, k, n, K) in enumerate(specs):
@@ -591,49 +590,54 @@ def bench_layer_stack(exl3, torch, peaks, stream, m):
     total_bytes = sum(layer_bytes(m, k, n, K) for (_nm, _m, k, n, K) in specs)
 
     names = [nm[len("70b_layer_"):].rsplit("_m", 1)[0] for (nm, _m, _k, _n, _K) in specs]
-    if use_gemv:
-        # one exl3_gemv_multi call per group of layers a decoder layer can run
-        # together: q/k/v share their input, so do gate/up; o, down and
-        # lm_head each wait for the layer before
-        groups = [["q", "k", "v"], ["o"], ["gate", "up"], ["down"], ["lm_head"]]
-        calls = []
-        for grp in groups:
-            idx = [names.index(g) for g in grp]
-            mc = exl3.GemvMulti([D[i] for i in idx])
-            calls.append((mc, exl3.new_workspace(mc.workspace_size)))
+    # one exl3_matmul_multi call per group of layers a decoder layer can run
+    # together (the GEMV multi call at m <= 16, the GEMM multi call above):
+    # q/k/v share their input, so do gate/up; o, down and lm_head each wait
+    # for the layer before
+    groups = [["q", "k", "v"], ["o"], ["gate", "up"], ["down"], ["lm_head"]]
+    calls = []
+    for grp in groups:
+        idx = [names.index(g) for g in grp]
+        mc = exl3.MultiCall([D[i] for i in idx], kind="matmul")
+        calls.append((mc, exl3.new_workspace(mc.workspace_size)))
 
-        def one_pass():
-            for mc, w in calls:
-                mc(w, stream=stream)
-    else:
-        def one_pass():
-            # the library picks the kernel (exl3_matmul: the GEMM for m > 16)
-            for x, t, suh, svh, K, y in D:
-                exl3.exl3_matmul(x, t, suh, svh, K, y=y, workspace=ws, stream=stream)
+    def one_pass():
+        for mc, w in calls:
+            mc(w, stream=stream)
 
-    with torch.cuda.stream(stream):
-        for _ in range(2):
-            one_pass()
-    stream.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream):
-        one_pass()
-    reps = 10
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            g.replay()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(reps):
-            g.replay()
-        e1.record(stream)
-    torch.cuda.synchronize()
-    us = e0.elapsed_time(e1) / reps * 1e3
-    del g
-    return {"workload": "llama3.1-70b decoder-layer linear stack + lm_head, m=%d (%s)" %
-                        (m, "exl3_gemv_multi per dependency group: q/k/v, o, gate/up, down, lm_head"
-                         if use_gemv else "exl3_matmul per layer, which runs the GEMM at this m"),
+    def per_layer_pass():
+        # the same layers as one exl3_matmul call each, for comparison
+        for x, t, suh, svh, K, y in D:
+            exl3.exl3_matmul(x, t, suh, svh, K, y=y, workspace=ws, stream=stream)
+
+    def graph_us(fn):
+        with torch.cuda.stream(stream):
+            for _ in range(2):
+                fn()
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+        reps = 10
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                g.replay()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        del g
+        return e0.elapsed_time(e1) / reps * 1e3
+
+    us = graph_us(one_pass)
+    us_single = graph_us(per_layer_pass)
+    return {"workload": "llama3.1-70b decoder-layer linear stack + lm_head, m=%d (exl3_matmul_multi per "
+                        "dependency group: q/k/v, o, gate/up, down, lm_head; the %s multi call at this m)" %
+                        (m, "GEMV" if m <= 16 else "GEMM"),
+            "us_per_pass_one_call_per_layer": us_single,
             "layers": [nm for (nm, _m, _k, _n, _K) in specs], "us_per_pass": us,
             "algorithmic_bytes_per_pass": total_bytes, "gb_s": total_bytes / (us * 1e-6) / 1e9,
             "frac_of_hbm_peak": total_bytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"]}

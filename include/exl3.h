@@ -212,6 +212,30 @@ exl3_status exl3_gemm(const void *x, const uint16_t *trellis, const void *suh, c
                       size_t workspace_bytes, void *stream);
 
 /*
+ * exl3_gemm_multi -- several layers with the same batch size m, the same k and
+ * the same K (each with its own x, suh, svh, y and n) through the tensor-core
+ * GEMM in one call: y_i = svh_i .* H(H(x_i .* suh_i) . W_hat_i).  ([GEMM]
+ * section GEMM内核: the kernel map picks the tiling for the shape; the layers
+ * of a decoder block that read the same activations -- q/k/v, gate/up -- are
+ * one problem with more output columns.)
+ *   layers    HOST array of `count` descriptors, as for exl3_gemv_multi.
+ *   count     1 .. any; every 8 layers (in call order) run as one rotation
+ *             launch and one persistent GEMM launch whose output tiles are
+ *             all the layers' tiles, so the stream-K split balances them
+ *             together (a narrow layer such as a k or v projection alone
+ *             would leave most of the GPU waiting on its few tiles).
+ *   workspace at least exl3_gemm_multi_workspace_size bytes (one tiled x' per
+ *             layer of a launch), zero-filled once after allocation, not
+ *             shared by concurrent calls.
+ * Results equal exl3_gemm's for each layer to within the stated tolerance.
+ * EXL3_ERR_INVALID_ARG if a descriptor is invalid, EXL3_ERR_UNSUPPORTED if
+ * the layers' k or K differ (nothing is launched in either case).
+ */
+size_t exl3_gemm_multi_workspace_size(const exl3_linear *layers, int count, int64_t m);
+exl3_status exl3_gemm_multi(const exl3_linear *layers, int count, int64_t m, void *workspace,
+                            size_t workspace_bytes, void *stream);
+
+/*
  * exl3_matmul -- the layer for any m >= 1 with the kernel chosen inside the
  * library ([GEMM] section GEMM内核: a kernel map picks the kernel from the
  * problem shape; section 小批量GEMV: the decode-phase small batches are
@@ -225,6 +249,17 @@ size_t exl3_matmul_workspace_size(int64_t m, int64_t k, int64_t n, int K);
 exl3_status exl3_matmul(const void *x, const uint16_t *trellis, const void *suh, const void *svh,
                         void *y, int64_t m, int64_t k, int64_t n, int K, void *workspace,
                         size_t workspace_bytes, void *stream);
+
+/*
+ * exl3_matmul_multi -- several layers with the same batch size m in one call,
+ * with the kernel chosen by m as for exl3_matmul: m <= 16 runs
+ * exl3_gemv_multi (any mix of k and K), larger m runs exl3_gemm_multi (all
+ * layers with the same k and K).  Workspace: exl3_matmul_multi_workspace_size
+ * bytes, zero-filled once after allocation.  Errors as the selected call.
+ */
+size_t exl3_matmul_multi_workspace_size(const exl3_linear *layers, int count, int64_t m);
+exl3_status exl3_matmul_multi(const exl3_linear *layers, int count, int64_t m, void *workspace,
+                              size_t workspace_bytes, void *stream);
 
 /*
  * exl3_encode -- tail-biting trellis encoding of a weight matrix: for every

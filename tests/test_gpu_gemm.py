@@ -138,3 +138,60 @@ def test_matmul_dispatch_matches_the_oracle(m):
     torch.cuda.synchronize()
     assert exl3.exl3_workspace_status(ws) == exl3.EXL3_OK
     check(layer, y.cpu().numpy().astype(np.float64))
+
+
+def _multi_layers(m, specs, seed):
+    """Layers of one multi call: each spec (k, n, K) gets its own x, trellis,
+    suh and svh."""
+    return [inputs.make_layer(m, k, n, K, seed=seed + i) for i, (k, n, K) in enumerate(specs)]
+
+
+def _multi_args(layers):
+    return [(dev(L.x), dev(L.trellis), dev(L.suh), dev(L.svh), L.K, None) for L in layers]
+
+
+@pytest.mark.parametrize("m,specs", [
+    (32, [(512, 1024, 3), (512, 256, 3), (512, 256, 3)]),              # q/k/v-like: one wide, two narrow
+    (40, [(256, 384, 2), (256, 128, 2)]),                              # half-width tiles in both layers
+    (200, [(384, 512, 4), (384, 640, 4), (384, 128, 4)]),              # weights-as-B form, ragged m
+    (17, [(1024, 256, 8)] * 3 + [(1024, 384, 8)] * 7),                 # 10 layers: two launches
+])
+def test_gemm_multi_matches_the_oracle(m, specs):
+    """exl3_gemm_multi: every layer's y equals the oracle's (each layer with its
+    own x, suh, svh; tiles of all layers share one launch's stream-K split)."""
+    layers = _multi_layers(m, specs, seed=7100 + m)
+    args = _multi_args(layers)
+    ws = exl3.new_workspace(exl3.exl3_gemm_multi_workspace_size(args, m))
+    ys = exl3.exl3_gemm_multi(args, workspace=ws)
+    torch.cuda.synchronize()
+    assert exl3.exl3_workspace_status(ws) == exl3.EXL3_OK
+    for L, y in zip(layers, ys):
+        check(L, y.cpu().numpy().astype(np.float64))
+    # a second call on the same workspace (counters back at zero) gives the same bits
+    ys2 = exl3.exl3_gemm_multi(args, workspace=ws)
+    torch.cuda.synchronize()
+    for y, y2 in zip(ys, ys2):
+        assert torch.equal(y, y2)
+
+
+def test_gemm_multi_rejects_mixed_k_or_K():
+    for specs in ([(256, 256, 3), (512, 256, 3)], [(256, 256, 3), (256, 256, 4)]):
+        args = _multi_args(_multi_layers(32, specs, seed=7300))
+        assert exl3.exl3_gemm_multi_workspace_size(args, 32) == 0
+        with pytest.raises(exl3.Exl3Error) as e:
+            exl3.exl3_gemm_multi(args, workspace=exl3.new_workspace(1 << 20))
+        assert e.value.status == exl3.EXL3_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("m", [8, 40])
+def test_matmul_multi_matches_the_oracle(m):
+    """exl3_matmul_multi: the GEMV multi call below m = 17 (any mix of k and K
+    is allowed there), the GEMM multi call above."""
+    specs = [(512, 384, 2), (512, 256, 2)] if m > 16 else [(512, 384, 2), (256, 256, 5)]
+    layers = _multi_layers(m, specs, seed=7400 + m)
+    args = _multi_args(layers)
+    ws = exl3.new_workspace(exl3.exl3_matmul_multi_workspace_size(args, m))
+    ys = exl3.exl3_matmul_multi(args, workspace=ws)
+    torch.cuda.synchronize()
+    for L, y in zip(layers, ys):
+        check(L, y.cpu().numpy().astype(np.float64))

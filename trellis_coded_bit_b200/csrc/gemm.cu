@@ -279,18 +279,34 @@ __device__ __forceinline__ void fwht32(float (&v)[32])
 
 // -------------------------------------------------------- rotation pass ---
 
-// x'[r, :] = H(x[r, :] .* suh)/sqrt(128) written in the tiled, swizzled A
-// layout: tile (r/128, c/64), 128-byte row r%128, 16-byte chunk ((c%64)/8) ^ (r%8).
-__global__ void __launch_bounds__(256) rotate_tiled_kernel(const __half *__restrict__ x,
-                                                           const __half *__restrict__ suh,
-                                                           unsigned char *__restrict__ xt, int m, int k)
+constexpr int kGemmMaxLayers = 8;  // layers per launch
+
+// The layers of one rotation launch (same m and k): x, suh and the tiled x'.
+struct GemmRotParams {
+    const __half *x[kGemmMaxLayers];
+    const __half *suh[kGemmMaxLayers];
+    unsigned char *xt[kGemmMaxLayers];
+    int nlayers, m, k;
+};
+
+// x'[r, :] = H(x[r, :] .* suh)/sqrt(128) of each layer written in the tiled,
+// swizzled A layout: tile (r/128, c/64), 128-byte row r%128, 16-byte chunk
+// ((c%64)/8) ^ (r%8).  A warp per (layer, row, 128-channel block).
+__global__ void __launch_bounds__(256) rotate_tiled_kernel(const GemmRotParams rp)
 {
     const int lane = threadIdx.x & 31;
     grid_dep_wait();    // x is produced by the preceding kernel
     grid_dep_launch();  // the GEMM kernel may set up (barriers, TMEM) meanwhile
-    const int64_t blocks = (int64_t)m * (k / 128);
+    const int m = rp.m, k = rp.k;
+    const int64_t per_layer = (int64_t)m * (k / 128);
+    const int64_t blocks = per_layer * rp.nlayers;
     const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < blocks; w += warps) {
+    for (int64_t wj = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); wj < blocks; wj += warps) {
+        const int l = (int)(wj / per_layer);
+        const int64_t w = wj - (int64_t)l * per_layer;
+        const __half *__restrict__ x = rp.x[l];
+        const __half *__restrict__ suh = rp.suh[l];
+        unsigned char *__restrict__ xt = rp.xt[l];
         const int r = (int)(w / (k / 128));
         const int blk = (int)(w - (int64_t)r * (k / 128));
         const int c = blk * 128 + lane * 4;
@@ -340,16 +356,24 @@ __device__ __forceinline__ void decode_row_to_b(const uint32_t *tile, int row, c
 
 // ------------------------------------------------------------ main kernel ---
 
-struct GemmParams {
-    const unsigned char *xt;   // tiled x'
+// One layer of a launch: its output columns are the launch's tile columns
+// [tn_begin, tn_begin + ceil(n / 256)); every layer has the launch's m, k, K.
+struct GemmLayer {
+    const unsigned char *xt;   // the layer's tiled x'
     const uint16_t *trellis;
     const __half *svh;
     __half *y;
+    int n, tn_begin;
+};
+
+struct GemmParams {
+    GemmLayer L[kGemmMaxLayers];
+    int nlayers;
     float *partials;           // [2 G][kPartialFloats] split-segment accumulators
     uint32_t *counters;        // [tiles] arrival tickets (return to zero)
     uint32_t *status;
-    int m, k, n;
-    int tiles_n;               // n / 256
+    int m, k;
+    int tiles_n;               // tile columns of all layers
     int kb_count;              // k / 64 units per tile
     uint32_t units;            // tiles * kb_count (units * ctas < 2^32)
     int ctas;                  // grid size G
@@ -368,6 +392,15 @@ struct GemmBars {
     int ticket;
 };
 static_assert(sizeof(GemmBars) <= 1024, "barrier block");
+
+// The layer that owns tile column tn.
+__device__ __forceinline__ int gemm_layer_of(const GemmParams &p, int tn)
+{
+    int l = 0;
+    while (l + 1 < p.nlayers && tn >= p.L[l + 1].tn_begin)
+        ++l;
+    return l;
+}
 
 // CTA owning unit u: the largest c with floor(c U / G) <= u.  (32-bit: the
 // host guarantees U * G < 2^32.)
@@ -504,7 +537,9 @@ __device__ __forceinline__ bool gemm_epilogue(const GemmParams &p, GemmBars &bar
         // row per instruction (8 rows per warp store instead of 32).
         // The last tile of n = 256j + 128 carries 128 columns: its other half
         // holds results of stale weights and is not stored.
-        const int halves = (tn + 1) * kBN > p.n ? 1 : kBN / 128;
+        const GemmLayer &L = p.L[gemm_layer_of(p, tn)];
+        const int tnl = tn - L.tn_begin;         // tile column within the layer
+        const int halves = (tnl + 1) * kBN > L.n ? 1 : kBN / 128;
         const int gi = lane & 3;                 // piece this lane stores
         const int grow = erow - gi;              // first row of the lane's group
         for (int mt = 0; mt < mt_count; ++mt) {
@@ -538,12 +573,12 @@ __device__ __forceinline__ bool gemm_epilogue(const GemmParams &p, GemmBars &bar
                     for (int i = 0; i < 32; ++i)
                         v[i] = __uint_as_float(r[i]);
                     fwht32(v);
-                    const int ncol0 = tn * kBN + hb * 128 + 32 * c;
+                    const int ncol0 = tnl * kBN + hb * 128 + 32 * c;
                     // piece q (columns 8q .. 8q + 7 of the chunk) as 4 words
                     uint32_t pc[4][4];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const uint4 sv4 = *reinterpret_cast<const uint4 *>(p.svh + ncol0 + 8 * q);
+                        const uint4 sv4 = *reinterpret_cast<const uint4 *>(L.svh + ncol0 + 8 * q);
                         const __half2 *sv = reinterpret_cast<const __half2 *>(&sv4);
                         const float sc = 0.08838834764831845f;
 #pragma unroll
@@ -577,7 +612,7 @@ __device__ __forceinline__ bool gemm_epilogue(const GemmParams &p, GemmBars &bar
 #pragma unroll
                     for (int sr = 0; sr < 4; ++sr)
                         if (row0 + sr < p.m)
-                            *reinterpret_cast<uint4 *>(p.y + (int64_t)(row0 + sr) * p.n + ncol0 + 8 * gi) =
+                            *reinterpret_cast<uint4 *>(L.y + (int64_t)(row0 + sr) * L.n + ncol0 + 8 * gi) =
                                 make_uint4(pc[sr][0], pc[sr][1], pc[sr][2], pc[sr][3]);
                 }
             }
@@ -682,7 +717,9 @@ __device__ __forceinline__ bool gemm_epilogue_wa(const GemmParams &p, GemmBars &
     }
     if (finish) {
         // the last tile of n = 256j + 128 carries only channel half 0
-        const int fchunks = (tn + 1) * kBN > p.n ? nchunks / 2 : nchunks;
+        const GemmLayer &L = p.L[gemm_layer_of(p, tn)];
+        const int tnl = tn - L.tn_begin;  // tile column within the layer
+        const int fchunks = (tnl + 1) * kBN > L.n ? nchunks / 2 : nchunks;
 #pragma unroll 1
         for (int cc = 0; cc < fchunks; ++cc) {
             const int h = (32 * cc) / nb, b0 = 32 * cc - h * nb;
@@ -692,8 +729,8 @@ __device__ __forceinline__ bool gemm_epilogue_wa(const GemmParams &p, GemmBars &
             for (int j = 0; j < 32; ++j)
                 ebuf[j * 128 + nrow] = __uint_as_float(r[j]);
             epi_sync();
-            const int ncol = tn * kBN + h * 128 + 4 * lane;
-            const uint2 sv2 = *reinterpret_cast<const uint2 *>(p.svh + ncol);
+            const int ncol = tnl * kBN + h * 128 + 4 * lane;
+            const uint2 sv2 = *reinterpret_cast<const uint2 *>(L.svh + ncol);
             const __half2 *sv = reinterpret_cast<const __half2 *>(&sv2);
 #pragma unroll 1
             for (int i = 0; i < 8; ++i) {
@@ -708,7 +745,7 @@ __device__ __forceinline__ bool gemm_epilogue_wa(const GemmParams &p, GemmBars &
                     uint2 out;
                     out.x = *reinterpret_cast<uint32_t *>(&o0);
                     out.y = *reinterpret_cast<uint32_t *>(&o1);
-                    *reinterpret_cast<uint2 *>(p.y + (int64_t)(b0 + j) * p.n + ncol) = out;
+                    *reinterpret_cast<uint2 *>(L.y + (int64_t)(b0 + j) * L.n + ncol) = out;
                 }
             }
             epi_sync();  // ebuf is refilled by the next chunk
@@ -783,6 +820,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmParams 
             int kb = (int)(u0 - t * KB);
             int tm = (int)(t / p.tiles_n);
             int mt_count = (p.m - tm * kBM * kMT) > kBM ? kMT : 1;  // skip an all-padding M tile
+            const unsigned char *xt = p.L[gemm_layer_of(p, (int)(t - (uint32_t)tm * p.tiles_n))].xt;
             int issued = 0;
             for (int i = 0; i < nu; ++i) {
                 const int s = i % kAStages;
@@ -795,12 +833,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmParams 
                 if constexpr (WA) {
                     // the first nb rows (batches) of x' tile (0, kb): nb x 128 contiguous bytes
                     mbar_arrive_expect_tx(&bars.afull[s], (uint32_t)(p.nb * 128));
-                    bulk_g2s(dst, p.xt + (int64_t)kb * kATileBytes, (uint32_t)(p.nb * 128), &bars.afull[s]);
+                    bulk_g2s(dst, xt + (int64_t)kb * kATileBytes, (uint32_t)(p.nb * 128), &bars.afull[s]);
                 } else {
                     mbar_arrive_expect_tx(&bars.afull[s], (uint32_t)(mt_count * kATileBytes));
                     for (int mt = 0; mt < mt_count; ++mt) {
                         const int64_t tile = (int64_t)(tm * kMT + mt) * (p.k / kBK) + kb;
-                        bulk_g2s(dst + mt * kATileBytes, p.xt + tile * kATileBytes, kATileBytes, &bars.afull[s]);
+                        bulk_g2s(dst + mt * kATileBytes, xt + tile * kATileBytes, kATileBytes, &bars.afull[s]);
                     }
                 }
                 issued = i + 1;
@@ -809,6 +847,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmParams 
                     ++t;
                     tm = (int)(t / p.tiles_n);
                     mt_count = (p.m - tm * kBM * kMT) > kBM ? kMT : 1;
+                    xt = p.L[gemm_layer_of(p, (int)(t - (uint32_t)tm * p.tiles_n))].xt;
                 }
             }
             for (int i = (issued > kAStages ? issued - kAStages : 0); i < issued; ++i)
@@ -821,7 +860,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmParams 
             uint32_t t = u0 / KB;
             int kb = (int)(u0 - t * KB);
             int tn = (int)(t % p.tiles_n);
-            const int64_t row_words = (int64_t)(p.n / 16) * 16 * K;  // one tile row of the matrix
+            // the tile column's layer: its trellis, a tile row of its matrix
+            // (row_words), the column within it and whether it is half width
+            const uint16_t *trel = nullptr;
+            int64_t row_words = 0;
+            int tnl = 0, row_bytes = kTileRowBytes;
+            auto enter_column = [&]() {
+                const GemmLayer &L = p.L[gemm_layer_of(p, tn)];
+                trel = L.trellis;
+                row_words = (int64_t)(L.n / 16) * 16 * K;
+                tnl = tn - L.tn_begin;
+                // the last tile of n = 256j + 128 has 8 trellis tiles per tile
+                // row, not 16; the decoders decode stale bytes for the rest
+                row_bytes = (tnl + 1) * kBN > L.n ? kTileRowBytes / 2 : kTileRowBytes;
+            };
+            enter_column();
             int issued = 0;
             for (int i = 0; i < nu; ++i) {
                 const int s = i % TS;
@@ -831,11 +884,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmParams 
                     break;
                 }
                 unsigned char *dst = tring + s * kTrBytes;
-                // the last tile of n = 256j + 128 has 8 trellis tiles per tile
-                // row, not 16; the decoders decode stale bytes for the rest
-                const int row_bytes = (tn + 1) * kBN > p.n ? kTileRowBytes / 2 : kTileRowBytes;
                 mbar_arrive_expect_tx(&bars.tfull[s], (uint32_t)((kBK / 16) * row_bytes));
-                const uint16_t *src = p.trellis + (int64_t)kb * (kBK / 16) * row_words + (int64_t)tn * 16 * 16 * K;
+                const uint16_t *src = trel + (int64_t)kb * (kBK / 16) * row_words + (int64_t)tnl * 16 * 16 * K;
 #pragma unroll
                 for (int r = 0; r < kBK / 16; ++r)
                     bulk_g2s(dst + r * kTileRowBytes, src + r * row_words, (uint32_t)row_bytes, &bars.tfull[s]);
@@ -844,6 +894,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmParams 
                     kb = 0;
                     ++t;
                     tn = (int)(t % p.tiles_n);
+                    enter_column();
                 }
             }
             for (int i = (issued > TS ? issued - TS : 0); i < issued; ++i)
@@ -985,14 +1036,21 @@ constexpr size_t kGemmSyncArea = 64 * 1024;
 struct GemmPlan {
     int64_t tiles, units;
     int tiles_n, kb_count, ctas;
-    size_t counters, xt, partials, total;  // workspace layout (byte offsets, total size)
+    size_t counters, xt, xt_bytes, partials, total;  // workspace layout (byte offsets, sizes)
 };
 
-static GemmPlan gemm_plan(int64_t m, int64_t k, int64_t n, int sms)
+// Plan of one launch over `count` layers with the same m, k and K and output
+// widths n[0..count): tile columns are the layers' in order (each n = 256j or
+// 256j + 128, whose last tile is half width).  Workspace: [0, 64 KB) status
+// word and one ticket per tile; then each layer's tiled x'; then two fp32
+// partial slots per CTA.
+static GemmPlan gemm_plan(int64_t m, int64_t k, const int64_t *n, int count, int sms)
 {
     GemmPlan pl;
     const int64_t tiles_m = (m + kBM * kMT - 1) / (kBM * kMT);
-    pl.tiles_n = (int)((n + kBN - 1) / kBN);  // n = 256j + 128: a half-width last tile
+    pl.tiles_n = 0;
+    for (int l = 0; l < count; ++l)
+        pl.tiles_n += (int)((n[l] + kBN - 1) / kBN);
     pl.tiles = tiles_m * pl.tiles_n;
     pl.kb_count = (int)(k / kBK);
     pl.units = pl.tiles * pl.kb_count;
@@ -1007,7 +1065,8 @@ static GemmPlan gemm_plan(int64_t m, int64_t k, int64_t n, int sms)
     // after every call of either kind, so one workspace can serve GEMV and
     // GEMM calls of any shapes in turn
     pl.xt = pl.xt > kGemmSyncArea ? pl.xt : kGemmSyncArea;
-    pl.partials = pl.xt + (size_t)(tiles_m * kBM * kMT) * (size_t)k * 2;
+    pl.xt_bytes = ((size_t)(tiles_m * kBM * kMT) * (size_t)k * 2 + 1023) / 1024 * 1024;
+    pl.partials = pl.xt + (size_t)count * pl.xt_bytes;
     pl.total = pl.partials + (size_t)2 * pl.ctas * kPartialFloats * 4;
     return pl;
 }
@@ -1026,47 +1085,55 @@ static exl3_status launch_gemm_t(const GemmParams &p, cudaStream_t stream)
 
 }  // namespace exl3
 
-extern "C" size_t exl3_gemm_workspace_size(int64_t m, int64_t k, int64_t n, int K)
-{
-    if (m < 1 || k < 128 || n < 128 || (k % 128) || (n % 128) || K < 1 || K > 8)
-        return 0;
-    return exl3::gemm_plan(m, k, n, exl3::num_sms()).total;
-}
+namespace exl3 {
 
-extern "C" exl3_status exl3_gemm(const void *x, const uint16_t *trellis, const void *suh,
-                                 const void *svh, void *y, int64_t m, int64_t k, int64_t n, int K,
-                                 void *workspace, size_t workspace_bytes, void *stream)
+// One rotation launch and one GEMM launch over `count` (1 .. kGemmMaxLayers)
+// layers with the same m, k and K, with the workspace laid out by gemm_plan.
+static exl3_status run_gemm_group(const exl3_linear *layers, int count, int64_t m, unsigned char *ws,
+                                  size_t ws_bytes, cudaStream_t s)
 {
-    using namespace exl3;
-    const exl3_status st = check_linear_args(x, trellis, suh, svh, y, m, k, n, K);
-    if (st != EXL3_OK)
-        return st;
-    const GemmPlan pl = gemm_plan(m, k, n, num_sms());
+    const int64_t k = layers[0].k;
+    const int K = layers[0].K;
+    int64_t n[kGemmMaxLayers];
+    for (int l = 0; l < count; ++l)
+        n[l] = layers[l].n;
+    const GemmPlan pl = gemm_plan(m, k, n, count, num_sms());
     if (pl.units * (int64_t)pl.ctas >= ((int64_t)1 << 32))
         return EXL3_ERR_UNSUPPORTED;  // split the call along m (about 10^14 multiply-adds per call)
-    if (!workspace || !aligned16(workspace) || workspace_bytes < pl.total)
+    if (!ws || !aligned16(ws) || ws_bytes < pl.total)
         return EXL3_ERR_WORKSPACE;
-    cudaStream_t s = (cudaStream_t)stream;
-    unsigned char *ws = (unsigned char *)workspace;
-    unsigned char *xt = ws + pl.xt;  // 16-byte aligned (1024-byte offset from an aligned base)
-    int64_t rot_grid = (m * (k / 128) + 7) / 8;
+    GemmRotParams rp;
+    rp.nlayers = count;
+    rp.m = (int)m;
+    rp.k = (int)k;
+    GemmParams p;
+    p.nlayers = count;
+    int tn = 0;
+    for (int l = 0; l < count; ++l) {
+        unsigned char *xt = ws + pl.xt + (size_t)l * pl.xt_bytes;  // 1024-byte offsets from an aligned base
+        rp.x[l] = (const __half *)layers[l].x;
+        rp.suh[l] = (const __half *)layers[l].suh;
+        rp.xt[l] = xt;
+        GemmLayer &L = p.L[l];
+        L.xt = xt;
+        L.trellis = layers[l].trellis;
+        L.svh = (const __half *)layers[l].svh;
+        L.y = (__half *)layers[l].y;
+        L.n = (int)n[l];
+        L.tn_begin = tn;
+        tn += (int)((n[l] + kBN - 1) / kBN);
+    }
+    int64_t rot_grid = (count * m * (k / 128) + 7) / 8;
     if (rot_grid > 148 * 16)
         rot_grid = 148 * 16;
-    if (launch_kernel(rotate_tiled_kernel, dim3((unsigned)rot_grid), dim3(256), 0, s, (const __half *)x,
-                      (const __half *)suh, xt, (int)m, (int)k) != cudaSuccess ||
+    if (launch_kernel(rotate_tiled_kernel, dim3((unsigned)rot_grid), dim3(256), 0, s, rp) != cudaSuccess ||
         launch_status() != EXL3_OK)
         return EXL3_ERR_CUDA;
-    GemmParams p;
-    p.xt = xt;
-    p.trellis = trellis;
-    p.svh = (const __half *)svh;
-    p.y = (__half *)y;
     p.partials = reinterpret_cast<float *>(ws + pl.partials);
     p.counters = reinterpret_cast<uint32_t *>(ws + pl.counters);
     p.status = (uint32_t *)ws;
     p.m = (int)m;
     p.k = (int)k;
-    p.n = (int)n;
     p.tiles_n = pl.tiles_n;
     p.kb_count = pl.kb_count;
     p.units = (uint32_t)pl.units;
@@ -1097,4 +1164,84 @@ extern "C" exl3_status exl3_gemm(const void *x, const uint16_t *trellis, const v
     case 7: return launch_gemm_t<7, false>(p, s);
     default: return launch_gemm_t<8, false>(p, s);
     }
+}
+
+// Argument checks of a multi call: every layer valid, and all with the first
+// layer's k and K (they share one launch's k loop and decode).
+static exl3_status check_gemm_multi(const exl3_linear *layers, int count, int64_t m)
+{
+    if (!layers || count < 1)
+        return EXL3_ERR_INVALID_ARG;
+    for (int l = 0; l < count; ++l) {
+        const exl3_linear &d = layers[l];
+        const exl3_status st = check_linear_args(d.x, d.trellis, d.suh, d.svh, d.y, m, d.k, d.n, d.K);
+        if (st != EXL3_OK)
+            return st;
+        if (d.k != layers[0].k || d.K != layers[0].K)
+            return EXL3_ERR_UNSUPPORTED;
+    }
+    return EXL3_OK;
+}
+
+}  // namespace exl3
+
+extern "C" size_t exl3_gemm_workspace_size(int64_t m, int64_t k, int64_t n, int K)
+{
+    if (m < 1 || k < 128 || n < 128 || (k % 128) || (n % 128) || K < 1 || K > 8)
+        return 0;
+    return exl3::gemm_plan(m, k, &n, 1, exl3::num_sms()).total;
+}
+
+extern "C" exl3_status exl3_gemm(const void *x, const uint16_t *trellis, const void *suh,
+                                 const void *svh, void *y, int64_t m, int64_t k, int64_t n, int K,
+                                 void *workspace, size_t workspace_bytes, void *stream)
+{
+    using namespace exl3;
+    const exl3_status st = check_linear_args(x, trellis, suh, svh, y, m, k, n, K);
+    if (st != EXL3_OK)
+        return st;
+    exl3_linear d;
+    d.x = x;
+    d.trellis = trellis;
+    d.suh = suh;
+    d.svh = svh;
+    d.y = y;
+    d.k = k;
+    d.n = n;
+    d.K = K;
+    return run_gemm_group(&d, 1, m, (unsigned char *)workspace, workspace_bytes, (cudaStream_t)stream);
+}
+
+extern "C" size_t exl3_gemm_multi_workspace_size(const exl3_linear *layers, int count, int64_t m)
+{
+    using namespace exl3;
+    if (check_gemm_multi(layers, count, m) != EXL3_OK)
+        return 0;
+    size_t most = 0;
+    for (int l0 = 0; l0 < count; l0 += kGemmMaxLayers) {
+        const int c = count - l0 < kGemmMaxLayers ? count - l0 : kGemmMaxLayers;
+        int64_t n[kGemmMaxLayers];
+        for (int l = 0; l < c; ++l)
+            n[l] = layers[l0 + l].n;
+        const size_t b = gemm_plan(m, layers[0].k, n, c, num_sms()).total;
+        most = b > most ? b : most;
+    }
+    return most;
+}
+
+extern "C" exl3_status exl3_gemm_multi(const exl3_linear *layers, int count, int64_t m, void *workspace,
+                                       size_t workspace_bytes, void *stream)
+{
+    using namespace exl3;
+    const exl3_status st = check_gemm_multi(layers, count, m);
+    if (st != EXL3_OK)
+        return st;
+    for (int l0 = 0; l0 < count; l0 += kGemmMaxLayers) {
+        const int c = count - l0 < kGemmMaxLayers ? count - l0 : kGemmMaxLayers;
+        const exl3_status rs =
+            run_gemm_group(layers + l0, c, m, (unsigned char *)workspace, workspace_bytes, (cudaStream_t)stream);
+        if (rs != EXL3_OK)
+            return rs;
+    }
+    return EXL3_OK;
 }

@@ -31,3 +31,17 @@ extern "C" exl3_status exl3_matmul(const void *x, const uint16_t *trellis, const
         return exl3_gemv(x, trellis, suh, svh, y, m, k, n, K, workspace, workspace_bytes, stream);
     return exl3_gemm(x, trellis, suh, svh, y, m, k, n, K, workspace, workspace_bytes, stream);
 }
+
+extern "C" size_t exl3_matmul_multi_workspace_size(const exl3_linear *layers, int count, int64_t m)
+{
+    return m <= exl3::kMatmulGemvMaxM ? exl3_gemv_multi_workspace_size(layers, count, m)
+                                      : exl3_gemm_multi_workspace_size(layers, count, m);
+}
+
+extern "C" exl3_status exl3_matmul_multi(const exl3_linear *layers, int count, int64_t m, void *workspace,
+                                         size_t workspace_bytes, void *stream)
+{
+    if (m >= 1 && m <= exl3::kMatmulGemvMaxM)
+        return exl3_gemv_multi(layers, count, m, workspace, workspace_bytes, stream);
+    return exl3_gemm_multi(layers, count, m, workspace, workspace_bytes, stream);
+}

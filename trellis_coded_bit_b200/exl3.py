@@ -26,6 +26,8 @@ EXPORTED = ["exl3_status_string", "exl3_version", "exl3_hadamard", "exl3_decode_
             "exl3_gemv_noalloc_max_scratch",
             "exl3_gemv_noalloc", "exl3_gemm_workspace_size", "exl3_gemm",
             "exl3_matmul_workspace_size", "exl3_matmul",
+            "exl3_gemm_multi_workspace_size", "exl3_gemm_multi",
+            "exl3_matmul_multi_workspace_size", "exl3_matmul_multi",
             "exl3_encode_workspace_size", "exl3_encode", "exl3_udu_workspace_size", "exl3_udu",
             "exl3_ldlq_workspace_size", "exl3_ldlq",
             "exl3_workspace_status", "exl3_set_launch_flags", "exl3_launch_flags",
@@ -80,10 +82,11 @@ def load(build_if_needed=True):
         for name in ("exl3_gemv", "exl3_gemm", "exl3_matmul"):
             getattr(lib, name).argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, ci, vp, sz, vp]
             getattr(lib, name).restype = ci
-        lib.exl3_gemv_multi_workspace_size.argtypes = [ctypes.POINTER(Exl3Linear), ci, i64]
-        lib.exl3_gemv_multi_workspace_size.restype = sz
-        lib.exl3_gemv_multi.argtypes = [ctypes.POINTER(Exl3Linear), ci, i64, vp, sz, vp]
-        lib.exl3_gemv_multi.restype = ci
+        for kind in ("gemv", "gemm", "matmul"):
+            getattr(lib, "exl3_%s_multi_workspace_size" % kind).argtypes = [ctypes.POINTER(Exl3Linear), ci, i64]
+            getattr(lib, "exl3_%s_multi_workspace_size" % kind).restype = sz
+            getattr(lib, "exl3_%s_multi" % kind).argtypes = [ctypes.POINTER(Exl3Linear), ci, i64, vp, sz, vp]
+            getattr(lib, "exl3_%s_multi" % kind).restype = ci
         lib.exl3_gemv_noalloc_max_scratch.argtypes = []
         lib.exl3_gemv_noalloc_max_scratch.restype = sz
         lib.exl3_gemv_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, ci, vp]
@@ -239,39 +242,82 @@ def _linear_array(layers, m):
     return arr, ys
 
 
+def _multi_workspace_size(kind, layers, m):
+    arr, _ = _linear_array(layers, m)
+    return int(getattr(load(), "exl3_%s_multi_workspace_size" % kind)(arr, len(layers), m))
+
+
+def _multi(kind, layers, workspace, stream):
+    m = layers[0][0].shape[0]
+    arr, ys = _linear_array(layers, m)
+    name = "exl3_%s_multi" % kind
+    if workspace is None:
+        raise ValueError("%s needs a workspace (%s_workspace_size)" % (name, name))
+    _check(getattr(load(), name)(arr, len(layers), m, _dev(workspace, torch.uint8, "workspace"),
+                                 workspace.numel(), _stream(stream)), name)
+    return ys
+
+
 def exl3_gemv_multi_workspace_size(layers, m):
     """Workspace bytes for exl3_gemv_multi over `layers` (see exl3_gemv_multi)."""
-    arr, _ = _linear_array(layers, m)
-    return int(load().exl3_gemv_multi_workspace_size(arr, len(layers), m))
+    return _multi_workspace_size("gemv", layers, m)
 
 
 def exl3_gemv_multi(layers, workspace=None, stream=None):
     """Several independent layers (same m <= 16) in one call: each entry is
     (x, trellis, suh, svh, K, y-or-None); returns the list of y."""
-    m = layers[0][0].shape[0]
-    arr, ys = _linear_array(layers, m)
-    if workspace is None:
-        raise ValueError("exl3_gemv_multi needs a workspace (exl3_gemv_multi_workspace_size)")
-    _check(load().exl3_gemv_multi(arr, len(layers), m, _dev(workspace, torch.uint8, "workspace"),
-                                  workspace.numel(), _stream(stream)), "exl3_gemv_multi")
-    return ys
+    return _multi("gemv", layers, workspace, stream)
 
 
-class GemvMulti:
-    """A prepared exl3_gemv_multi call: the descriptor array is built once, so
-    repeated calls (a decode loop) cost only the C call.  `layers` as for
-    exl3_gemv_multi; the tensors must stay alive and in place."""
+def exl3_gemm_multi_workspace_size(layers, m):
+    """Workspace bytes for exl3_gemm_multi over `layers` (see exl3_gemm_multi)."""
+    return _multi_workspace_size("gemm", layers, m)
 
-    def __init__(self, layers):
+
+def exl3_gemm_multi(layers, workspace=None, stream=None):
+    """Several layers with the same m, k and K through the GEMM in one call
+    (entries as for exl3_gemv_multi); returns the list of y."""
+    return _multi("gemm", layers, workspace, stream)
+
+
+def exl3_matmul_multi_workspace_size(layers, m):
+    """Workspace bytes for exl3_matmul_multi over `layers`."""
+    return _multi_workspace_size("matmul", layers, m)
+
+
+def exl3_matmul_multi(layers, workspace=None, stream=None):
+    """Several layers with the same m, the kernel chosen by m (GEMV multi for
+    m <= 16, GEMM multi above); returns the list of y."""
+    return _multi("matmul", layers, workspace, stream)
+
+
+class MultiCall:
+    """A prepared multi-layer call (`kind` "gemv", "gemm" or "matmul"): the
+    descriptor array is built once, so repeated calls (a decode loop) cost
+    only the C call.  `layers` as for exl3_gemv_multi; the tensors must stay
+    alive and in place."""
+
+    kind = "matmul"
+
+    def __init__(self, layers, kind=None):
+        if kind is not None:
+            self.kind = kind
         self.m = layers[0][0].shape[0]
         self.count = len(layers)
         self._arr, self.ys = _linear_array(layers, self.m)
-        self.workspace_size = int(load().exl3_gemv_multi_workspace_size(self._arr, self.count, self.m))
+        self._name = "exl3_%s_multi" % self.kind
+        self.workspace_size = int(getattr(load(), self._name + "_workspace_size")(self._arr, self.count, self.m))
 
     def __call__(self, workspace, stream=None):
-        _check(load().exl3_gemv_multi(self._arr, self.count, self.m, _dev(workspace, torch.uint8, "workspace"),
-                                      workspace.numel(), _stream(stream)), "exl3_gemv_multi")
+        _check(getattr(load(), self._name)(self._arr, self.count, self.m, _dev(workspace, torch.uint8, "workspace"),
+                                           workspace.numel(), _stream(stream)), self._name)
         return self.ys
+
+
+class GemvMulti(MultiCall):
+    """A prepared exl3_gemv_multi call (see MultiCall)."""
+
+    kind = "gemv"
 
 
 def exl3_gemv_noalloc_max_scratch():
