@@ -180,6 +180,39 @@ def test_gemv_llama70b_small_batch_sampled(case):
     check_layer(layer, y, col_blocks=(nb - 1, nb))
 
 
+# Where the GEMV's input rotation runs follows from the plan: inside the main
+# kernel (each CTA rotates the blocks its own units read) when every CTA's
+# unit range is at most the smallest tile-row count k/16 of its K group and
+# (range/8 + 2) * m <= 16; otherwise in a rotation kernel launched just
+# before.  The shapes below fall on both sides (ranges from the plan's grid:
+# min(296, units/16) CTAs, aligned to whole column blocks for one layer).
+@pytest.mark.parametrize("m,k,n,K,where", [
+    (1, 4096, 4096, 4, "in kernel"),          # 8192 units / 288 CTAs: 29 rows of 256
+    (4, 1024, 1024, 3, "in kernel"),          # 512 units / 32 CTAs: 16 rows of 64, 16 jobs per CTA
+    (16, 1024, 1024, 3, "separate"),          # the same ranges, 64 jobs per CTA
+    (1, 256, 38016, 2, "separate"),           # 297 column blocks: ranges of 17 > 16 tile rows
+])
+def test_gemv_rotation_in_kernel_or_separate(m, k, n, K, where):
+    layer = inputs.make_layer(m, k, n, K, seed=7600 + m + K)
+    y, _ = run_gemv(layer)
+    nb = n // 128
+    check_layer(layer, y, col_blocks=(0, min(nb, 4)))
+    check_layer(layer, y, col_blocks=(nb - 2, nb))
+
+
+def test_gemv_multi_in_kernel_rotation_across_layers():
+    # two layers of one K group, 360 units on 22 CTAs: ranges of 16-17 units
+    # (<= 24 tile rows), so each CTA rotates its own blocks, and CTA 14's range
+    # [229, 245) ends layer 0 (rows 13..23 of its last column block) and starts
+    # layer 1 (rows 0..4 of its first)
+    layers = [inputs.make_layer(1, 384, 1280, 3, seed=7700), inputs.make_layer(1, 384, 640, 3, seed=7701)]
+    args = [(dev(L.x), dev(L.trellis), dev(L.suh), dev(L.svh), L.K, None) for L in layers]
+    ws = exl3.new_workspace(exl3.exl3_gemv_multi_workspace_size(args, 1))
+    ys = exl3.exl3_gemv_multi(args, workspace=ws)
+    for L, y in zip(layers, ys):
+        check_layer(L, host(y).astype(np.float64))
+
+
 def test_gemm_timeout_reports_status_without_hang():
     # the GEMM's stage hand-offs are bounded waits: with a 1 ns bound they run
     # out, the kernel records EXL3_ERR_TIMEOUT and returns -- no fault, no hang
