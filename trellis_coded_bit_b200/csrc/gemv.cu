@@ -747,11 +747,12 @@ struct GemvPlan {
 
 // Relative time of one unit at m = 1 by K: each K group of the Llama-3.1-8B
 // decode set timed alone on B200, less about 8.5 us of fixed launch cost (K =
-// 1, 5, 7 interpolated; odd K load their runs in 4-byte pieces, larger K move
-// more bytes).  It sets each group's share of the grid.
+// 1, 5, 7 interpolated; K = 4 and 8 load their runs in 16-byte pieces and have
+// the cheapest windows, odd K load 4-byte pieces).  It sets each group's share
+// of the grid.
 static int64_t gemv_unit_cost(int K)
 {
-    static const int64_t cost[9] = {0, 300, 306, 327, 326, 345, 359, 371, 383};
+    static const int64_t cost[9] = {0, 296, 301, 323, 306, 335, 346, 336, 326};
     return cost[K < 1 ? 1 : (K > 8 ? 8 : K)];
 }
 
