@@ -227,9 +227,11 @@ exl3_status exl3_gemm(const void *x, const uint16_t *trellis, const void *suh, c
  *   workspace at least exl3_gemm_multi_workspace_size bytes (one tiled x' per
  *             layer of a launch), zero-filled once after allocation, not
  *             shared by concurrent calls.
- * Results equal exl3_gemm's for each layer to within the stated tolerance.
- * EXL3_ERR_INVALID_ARG if a descriptor is invalid, EXL3_ERR_UNSUPPORTED if
- * the layers' k or K differ (nothing is launched in either case).
+ * Layers must not write one another's inputs (x, trellis, suh, svh) and
+ * their y must not overlap.  Results equal exl3_gemm's for each layer to
+ * within the stated tolerance.  EXL3_ERR_INVALID_ARG if a descriptor is
+ * invalid, EXL3_ERR_UNSUPPORTED if the layers' k or K differ (nothing is
+ * launched in either case).
  */
 size_t exl3_gemm_multi_workspace_size(const exl3_linear *layers, int count, int64_t m);
 exl3_status exl3_gemm_multi(const exl3_linear *layers, int count, int64_t m, void *workspace,
