@@ -162,6 +162,44 @@ def test_gemv_multi_argument_errors_and_sizes():
     assert size([(A, B, C, D, E, 200, 256, 4)]) == 0
 
 
+def _gemm_multi(descs, m=32, ws=None, wsb=1 << 30, fn="exl3_gemm_multi"):
+    lib = exl3.load()
+    arr = (exl3.Exl3Linear * max(1, len(descs)))(*[exl3.Exl3Linear(*d) for d in descs])
+    return getattr(lib, fn)(arr, len(descs), m, ws, wsb, None)
+
+
+def test_gemm_multi_argument_errors_and_sizes():
+    lib = exl3.load()
+    good = (A, B, C, D, E, 256, 256, 4)
+    inv, uns = exl3.EXL3_ERR_INVALID_ARG, exl3.EXL3_ERR_UNSUPPORTED
+    assert _gemm_multi([]) == inv                                       # no layers
+    assert _gemm_multi([good, (A, B, C, D, E, 200, 256, 4)]) == inv     # one bad layer
+    assert _gemm_multi([good, (A, B, C, D, E, 512, 256, 4)]) == uns     # k differs
+    assert _gemm_multi([good, (A, B, C, D, E, 256, 256, 3)]) == uns     # K differs
+    assert _gemm_multi([good]) == exl3.EXL3_ERR_WORKSPACE               # no workspace
+    assert _gemm_multi([good], ws=A, wsb=16) == exl3.EXL3_ERR_WORKSPACE
+
+    def size(descs, m=32, kind="gemm"):
+        arr = (exl3.Exl3Linear * len(descs))(*[exl3.Exl3Linear(*d) for d in descs])
+        return getattr(lib, "exl3_%s_multi_workspace_size" % kind)(arr, len(descs), m)
+
+    one = size([good])
+    assert one == lib.exl3_gemm_workspace_size(32, 256, 256, 4)
+    # one tiled x' per layer of a launch: a second layer needs at least one more
+    wide = (A, B, C, D, E, 256, 1152, 4)
+    assert size([good, wide]) >= one + 32 * 256 * 2
+    # more than 8 layers run as several launches on the same workspace: the
+    # size is the largest launch's
+    assert size([good] * 9) == size([good] * 8)
+    assert size([good, (A, B, C, D, E, 256, 256, 5)]) == 0
+    # the matmul multi call picks by m
+    assert size([good], m=16, kind="matmul") == size([good], m=16, kind="gemv")
+    assert size([good], m=17, kind="matmul") == size([good], m=17, kind="gemm")
+    assert _gemm_multi([good, (A, B, C, D, E, 512, 256, 2)], m=8, fn="exl3_matmul_multi") == \
+        exl3.EXL3_ERR_WORKSPACE  # GEMV multi: any mix of k and K, only the workspace is missing
+    assert _gemm_multi([good, (A, B, C, D, E, 512, 256, 2)], m=40, fn="exl3_matmul_multi") == uns
+
+
 def test_encode_argument_errors_and_sizes():
     lib = exl3.load()
     inv = exl3.EXL3_ERR_INVALID_ARG
