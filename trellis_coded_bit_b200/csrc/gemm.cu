@@ -10,6 +10,11 @@
 //      it as fp16 directly in the tensor core's canonical K-major, 128-byte
 //      swizzled tile layout ([m/128][k/64] tiles of 128 rows x 64 channels,
 //      16 KB each), so one 1-D bulk copy moves one A tile into shared memory.
+//      A launch may serve up to 8 layers with the same m, k and K
+//      (exl3_gemm_multi: q/k/v, gate/up): each has its own x' region, and the
+//      GEMM's output tile columns are all the layers' columns in order (a
+//      small table gives each layer's x', trellis, svh, y, n and first tile
+//      column), so the stream-K split below balances them together.
 //   2. The main kernel is persistent and "stream-K" balanced: the work units
 //      are (256 x 256 output tile, 64-channel k block) pairs in tile order,
 //      and CTA c of G (G <= one per SM) owns units [cU/G, (c+1)U/G), so every
